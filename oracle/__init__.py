@@ -1,0 +1,20 @@
+"""Oracle for the QLoRA NF4 linear layer -- TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, obviously correct CPU restatement of what the GPU library computes, in fp64 wherever the
+method leaves the precision open.  It shares no code, table or constant with the CUDA library and imports
+nothing from it.  Only the test suite, the package's ``smoke()`` check and the CPU-baseline leg of the
+benchmark may import it; the product path never does.
+
+Modules
+-------
+``oracle.nf4``     NF4 codebook, blockwise quantize / dequantize, bf16 round-to-nearest-even.
+``oracle.linear``  forward / backward of the QLoRA linear layer, SwiGLU, and the gated-MLP chain.
+
+Pins: every function here is checked by ``tests/test_oracle_*.py`` against values fixed by the
+mathematics (closed forms, invariants, brute force on tiny inputs, finite differences, library routines
+for the special cases that reduce to them).  The one part with no external pin is the exact NF4 table:
+the pages name the level set but print no table ("parity unpinned" against the pages for the table
+values; see ``oracle.nf4.nf4_codebook``).
+"""
+
+from . import nf4, linear  # noqa: F401

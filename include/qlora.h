@@ -1,0 +1,178 @@
+/*
+ * qlora.h -- C ABI of libqlora, the B200 (sm_100a) QLoRA NF4 linear layer.
+ *
+ * The layer (per "Unsloth v0.1.463-beta: Fixes Studio Crash and llama-server Permission Issue",
+ * kongchang.com, section "About the Unsloth Project", paragraph "How LoRA and QLoRA work"; "unsloth",
+ * pyshine.com, section "Why You Need This"; "Inside Unsloth: How the Fastest LLM Fine-Tuning Library
+ * Works", thriftbooks.com, section "What You'll Learn", item "LoRA and QLoRA"):
+ *
+ *     y  = x deq(W)^T + s (x A^T) B^T                      forward
+ *     dX = dY deq(W) + s (dY B) A,  dA = s (dY B)^T x,  dB = s dY^T (x A^T)      backward (W frozen)
+ *
+ * with x [M,K] bf16 activations, W [N,K] stored as blockwise NF4 (4-bit codes + one fp32 absmax per
+ * 64-element block), LoRA adapters A [r,K] and B [N,r] in bf16 and the scaling s = lora_alpha / r.
+ *
+ * Conventions for every entry point
+ *   - Matrices are row-major and contiguous.  "bf16" buffers hold bfloat16 bit patterns (uint16_t).
+ *   - All data pointers are DEVICE pointers, 16-byte aligned.  The caller owns every buffer; the library
+ *     never allocates, frees or synchronizes (except ql_get_device_error, which says so).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls are asynchronous.
+ *   - Argument errors are detected on the host before any launch and return QL_ERR_INVALID_ARG (or
+ *     QL_ERR_UNSUPPORTED for valid but unimplemented parameters); nothing is launched then.  A failed
+ *     launch returns QL_ERR_CUDA.  Faults detected on the device (a bounded wait that gave up, a
+ *     non-finite block maximum) are latched in a device error word read by ql_get_device_error.
+ *   - The library keeps no state between calls apart from per-device constants (the NF4 table).
+ *   - Entry points need the CUDA device of `stream` to be current.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QL_API __attribute__((visibility("default")))
+#else
+#define QL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1,  /* bad shape, null or misaligned pointer, too-small workspace */
+  QL_ERR_UNSUPPORTED = 2,  /* valid parameters this build does not implement (e.g. blocksize != 64) */
+  QL_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
+  QL_ERR_TIMEOUT = 4       /* a kernel's bounded wait expired (reported by ql_get_device_error) */
+} ql_status;
+
+typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
+typedef enum { QL_PASS_FWD = 0, QL_PASS_BWD = 1 } ql_pass;
+
+/* Human-readable name of a status code (static string). */
+QL_API const char* ql_status_string(int status);
+
+/* ABI version of this library (incremented on incompatible changes). */
+QL_API int ql_abi_version(void);
+
+/* Copies the library's 16-entry NF4 level table (fp32, ascending) into host memory `out`.
+ * Host-only; needs no GPU.  The table follows the normal-quantile rule (8 positive and 7 negative
+ * standard-normal quantiles normalised to [-1, 1], plus an exact 0 at index 7). */
+QL_API void ql_nf4_codebook(float out[16]);
+
+/* Reads and clears the device error word of the current device after synchronizing `stream`.
+ * Returns QL_OK, QL_ERR_TIMEOUT (a kernel's bounded wait expired), QL_ERR_INVALID_ARG (nf4_quantize met
+ * a non-finite block), or QL_ERR_CUDA.  This is the only entry point that synchronizes. */
+QL_API ql_status ql_get_device_error(void* stream);
+
+/* Number of kernels this library has launched in the process so far (all devices).  Host-only. */
+QL_API uint64_t ql_launch_count(void);
+
+/* Observability hook.  `which` = 0: the fused forward GEMM of qlora_linear_fwd; 1: the fused dX GEMM of
+ * qlora_linear_bwd.  When `start`/`stop` (cudaEvent_t as void*) are non-NULL the library records them on
+ * the call's stream immediately before and after that one kernel; NULL disables.  Process-wide setting;
+ * the events stay owned by the caller.  Returns QL_ERR_INVALID_ARG for an unknown `which`. */
+QL_API ql_status ql_set_profile_events(int which, void* start, void* stop);
+
+/* Failure-detection self-test: launches one tiny kernel that waits on an mbarrier nobody arrives on, with
+ * the same bounded-wait code the GEMM kernels use but a limit of `wait_cycles` clock cycles (1 .. 2^32).
+ * The wait gives up, latches the timeout bit in the device error word and the kernel returns normally;
+ * ql_get_device_error then reports QL_ERR_TIMEOUT and the context stays usable. */
+QL_API ql_status ql_selftest_wait_timeout(int64_t wait_cycles, void* stream);
+
+/*
+ * nf4_quantize -- blockwise NF4 quantization of a frozen base weight ("How LoRA and QLoRA work", as above).
+ *   w        [numel] fp32, the flat row-major weight (W [N,K] gives numel = N*K).
+ *   numel    number of elements; a positive multiple of `blocksize`.
+ *   blocksize elements per absmax block; only 64 is supported (QL_ERR_UNSUPPORTED otherwise).
+ *   codes    [numel/2] uint8 out: element 2j in the HIGH nibble of byte j, element 2j+1 in the low nibble.
+ *   absmax   [numel/blocksize] fp32 out: max |w| of each block.
+ * Per block: n = w / absmax in IEEE fp32; code = number of level midpoints strictly below n (a value on
+ * a midpoint takes the lower code); an all-zero block stores absmax 0 and code 7 everywhere.  Bit-exact
+ * and deterministic.  Non-finite weights are outside the domain: the device error word records them.
+ */
+QL_API ql_status nf4_quantize(const float* w, int64_t numel, int blocksize, uint8_t* codes, float* absmax,
+                       void* stream);
+
+/*
+ * nf4_dequantize -- w' = fl32(level[code] * absmax) ("unsloth", pyshine.com, section "Why You Need This":
+ * NF4 weights dequantized on the fly; here materialized for checking and export).
+ *   codes, absmax  as produced by nf4_quantize; numel, blocksize as there.
+ *   out_dtype      QL_F32: out is float[numel] holding w';  QL_BF16: out is bf16[numel] holding
+ *                  round-to-nearest-even(w').
+ * Bit-exact and deterministic.
+ */
+QL_API ql_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t numel, int blocksize,
+                         ql_dtype out_dtype, void* out, void* stream);
+
+/*
+ * qlora_workspace_bytes -- device scratch needed by qlora_linear_fwd (pass = QL_PASS_FWD) or
+ * qlora_linear_bwd (QL_PASS_BWD) for these sizes on the current device (split-K partial sums, the
+ * rank-r intermediates s*x*A^T and s*dY*B).  Host-only.  Returns 0 when nothing is needed.
+ */
+QL_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass);
+
+/*
+ * qlora_linear_fwd -- y = x deq(W)^T + s (x A^T) B^T in one fused pass over the NF4 weight
+ * ("Inside Unsloth ...", section "What You'll Learn", item "LoRA and QLoRA": NF4 dequantization, matrix
+ * multiplication and LoRA correction fused; "unsloth", pyshine.com: the LoRA matmul that fuses the base
+ * quantized weight and the adapter delta into one call, and the dequantize-on-the-fly GEMV for small M).
+ *   M, N, K, r  x [M,K], W [N,K], A [r,K], B [N,r], y [M,N].  M >= 0; N >= 1 with N % 8 == 0;
+ *               K >= 64 with K % 64 == 0; 0 <= r <= 256 with r % 8 == 0 (r = 0: plain NF4 layer, A/B unused).
+ *   x           bf16 [M,K].
+ *   codes, absmax  NF4 weight from nf4_quantize of W (blocksize 64).
+ *   A, B        bf16 LoRA adapters.
+ *   s           LoRA scaling (lora_alpha / r).
+ *   y           bf16 [M,N] out (round-to-nearest-even of the fp32 accumulator).
+ *   su_out      nullable bf16 [M,r] out: s * x A^T rounded to bf16, the rank-r term the product uses;
+ *               pass it to qlora_linear_bwd to skip recomputing it.
+ *   workspace, ws_bytes  device scratch of at least qlora_workspace_bytes(M,N,K,r,QL_PASS_FWD) bytes
+ *               (may be NULL when that is 0).
+ * Products run on the tensor cores in bf16 with fp32 accumulation; deq(W) is formed in shared memory
+ * tile by tile and never written to global memory.  The result is deterministic for given sizes.
+ */
+QL_API ql_status qlora_linear_fwd(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x, const uint8_t* codes,
+                           const float* absmax, const uint16_t* A, const uint16_t* B, float s, uint16_t* y,
+                           uint16_t* su_out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * qlora_linear_bwd -- gradients of the layer with the base weight frozen ("How LoRA and QLoRA work": only
+ * the adapters train; "Unsloth v0.1.47-beta ..." (kongchang.com), section on LoRA/QLoRA: the rewritten
+ * backward keeps numerical equivalence).
+ *   dy          bf16 [M,N] upstream gradient.
+ *   x, codes, absmax, A, B, s   as in the forward (same size rules).
+ *   su          nullable bf16 [M,r]: the forward's su_out; recomputed when NULL.
+ *   dx          nullable bf16 [M,K] out: dY deq(W) + s (dY B) A.
+ *   dA          nullable fp32 [r,K] out: s (dY B)^T x.
+ *   dB          nullable fp32 [N,r] out: s dY^T (x A^T).
+ *   workspace, ws_bytes  at least qlora_workspace_bytes(M,N,K,r,QL_PASS_BWD) bytes.
+ * deq(W)^T tiles are formed in shared memory on the fly (never in global memory).  M = 0 writes dA = 0
+ * and dB = 0.  Deterministic for given sizes.
+ */
+QL_API ql_status qlora_linear_bwd(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* dy, const uint16_t* x,
+                           const uint8_t* codes, const float* absmax, const uint16_t* A, const uint16_t* B,
+                           float s, const uint16_t* su, uint16_t* dx, float* dA, float* dB, void* workspace,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * qlora_swiglu_fwd -- h = silu(g) * u elementwise, silu(g) = g / (1 + exp(-g)), in fp32, h rounded to
+ * bf16 ("Inside Unsloth ...", section "What You'll Learn", item "Triton Kernel Internals": the fused
+ * SwiGLU; "unsloth", pyshine.com: swiglu.py fuses the gated MLP activation).
+ *   numel >= 0; g, u, h bf16 [numel].
+ */
+QL_API ql_status qlora_swiglu_fwd(int64_t numel, const uint16_t* g, const uint16_t* u, uint16_t* h, void* stream);
+
+/*
+ * qlora_swiglu_bwd -- dg = dh * u * sigma(g) (1 + g (1 - sigma(g))), du = dh * silu(g), in fp32, rounded
+ * to bf16.  numel >= 0; all buffers bf16 [numel].  dg/du may alias dh (read before write per element).
+ */
+QL_API ql_status qlora_swiglu_bwd(int64_t numel, const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,
+                           uint16_t* du, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

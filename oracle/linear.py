@@ -63,14 +63,22 @@ def qlora_forward(x, Wd, A, B, s: float) -> np.ndarray:
     return x @ _f64(Wd).T + float(s) * (lora_down(x, A) @ _f64(B).T)
 
 
+def lora_grads(dy, x, A, B, s: float):
+    """(dA [r,K], dB [N,r]): the adapter gradients, which do not involve the base weight."""
+    dy, x, A, B = _f64(dy), _f64(x), _f64(A), _f64(B)
+    s = float(s)
+    v = dy @ B                      # dY B   [M,r]
+    dA = s * (v.T @ x)
+    dB = s * (dy.T @ (x @ A.T))
+    return dA, dB
+
+
 def qlora_backward(dy, x, Wd, A, B, s: float):
     """(dX [M,K], dA [r,K], dB [N,r]) of the forward above, for the upstream gradient dY [M,N]."""
     dy, x, Wd, A, B = _f64(dy), _f64(x), _f64(Wd), _f64(A), _f64(B)
     s = float(s)
-    v = dy @ B                      # dY B   [M,r]
-    dx = dy @ Wd + s * (v @ A)
-    dA = s * (v.T @ x)
-    dB = s * (dy.T @ (x @ A.T))
+    dx = dy @ Wd + s * ((dy @ B) @ A)
+    dA, dB = lora_grads(dy, x, A, B, s)
     return dx, dA, dB
 
 

@@ -1,0 +1,152 @@
+// Memory-bound kernels of the QLoRA layer: NF4 quantize / dequantize, split-K reduction, SwiGLU.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "nf4_table.cuh"
+#include "ptx.cuh"
+
+namespace qlora {
+
+// Midpoints between adjacent levels, exact in fp64 (a sum of two fp32 values and a halving).
+__constant__ double kNF4Mid[15] = {
+    (double(kNF4Levels[0]) + double(kNF4Levels[1])) * 0.5,   (double(kNF4Levels[1]) + double(kNF4Levels[2])) * 0.5,
+    (double(kNF4Levels[2]) + double(kNF4Levels[3])) * 0.5,   (double(kNF4Levels[3]) + double(kNF4Levels[4])) * 0.5,
+    (double(kNF4Levels[4]) + double(kNF4Levels[5])) * 0.5,   (double(kNF4Levels[5]) + double(kNF4Levels[6])) * 0.5,
+    (double(kNF4Levels[6]) + double(kNF4Levels[7])) * 0.5,   (double(kNF4Levels[7]) + double(kNF4Levels[8])) * 0.5,
+    (double(kNF4Levels[8]) + double(kNF4Levels[9])) * 0.5,   (double(kNF4Levels[9]) + double(kNF4Levels[10])) * 0.5,
+    (double(kNF4Levels[10]) + double(kNF4Levels[11])) * 0.5, (double(kNF4Levels[11]) + double(kNF4Levels[12])) * 0.5,
+    (double(kNF4Levels[12]) + double(kNF4Levels[13])) * 0.5, (double(kNF4Levels[13]) + double(kNF4Levels[14])) * 0.5,
+    (double(kNF4Levels[14]) + double(kNF4Levels[15])) * 0.5,
+};
+
+// Code of a normalised value: binary search for the number of midpoints strictly below n (exact fp64
+// comparisons; a value equal to a midpoint counts that midpoint as not below, so ties take the lower code).
+__device__ __forceinline__ uint32_t nf4_code(float n) {
+  const double v = static_cast<double>(n);
+  uint32_t lo = 0;  // answer in [0, 15]
+#pragma unroll
+  for (uint32_t step = 8; step > 0; step >>= 1) {
+    // invariant: midpoints [0, lo) are below v; test midpoint lo + step - 1
+    if (lo + step <= 15 && v > kNF4Mid[lo + step - 1]) lo += step;
+  }
+  return lo;
+}
+
+// One warp per 64-element block: lane l owns elements 2l, 2l+1 (one packed byte).
+__global__ void nf4_quantize_kernel(const float* __restrict__ w, long long nblocks, uint8_t* __restrict__ codes,
+                                    float* __restrict__ absmax, unsigned int* err) {
+  const int lane = threadIdx.x & 31;
+  const long long warps_total = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long b = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); b < nblocks;
+       b += warps_total) {
+    const float2 v = __ldg(reinterpret_cast<const float2*>(w) + b * 32 + lane);
+    float m = fmaxf(fabsf(v.x), fabsf(v.y));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const bool bad = !isfinite(v.x) || !isfinite(v.y);
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, kDevErrNonFinite);
+    uint32_t c0 = 7, c1 = 7;
+    if (m > 0.0f) {
+      c0 = nf4_code(__fdiv_rn(v.x, m));
+      c1 = nf4_code(__fdiv_rn(v.y, m));
+    }
+    codes[b * 32 + lane] = static_cast<uint8_t>((c0 << 4) | c1);
+    if (lane == 0) absmax[b] = m;
+  }
+}
+
+// Each thread expands 8 elements (4 code bytes) with one absmax.
+template <bool kBf16>
+__global__ void nf4_dequantize_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ absmax,
+                                      long long ngroups, void* __restrict__ out) {
+  __shared__ float lv[16];
+  if (threadIdx.x < 16) lv[threadIdx.x] = kNF4LevelsDev[threadIdx.x];
+  __syncthreads();
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
+    const uint32_t wv = __ldg(reinterpret_cast<const uint32_t*>(codes) + g);
+    const float sc = __ldg(absmax + (g >> 3));  // 8 groups of 8 per 64-element block
+    float f[8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t byte = (wv >> (8 * b)) & 0xFFu;
+      f[2 * b] = __fmul_rn(lv[byte >> 4], sc);
+      f[2 * b + 1] = __fmul_rn(lv[byte & 15u], sc);
+    }
+    if (kBf16) {
+      uint4 o;
+      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * b], f[2 * b + 1]);
+        op[b] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(out)[g] = o;
+    } else {
+      float4* o = reinterpret_cast<float4*>(out) + 2 * g;
+      o[0] = make_float4(f[0], f[1], f[2], f[3]);
+      o[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+  }
+}
+
+// out[e] = alpha * sum_s ws[s * slab + e]  (fp32 sum in split order: deterministic)
+__global__ void reduce_splits_kernel(const float* __restrict__ ws, long long slab, int nsplit, long long count,
+                                     float alpha, void* __restrict__ out, int out_bf16) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < count; e += stride) {
+    float acc = 0.0f;
+    for (int s = 0; s < nsplit; ++s) acc += ws[s * slab + e];
+    acc *= alpha;
+    if (out_bf16)
+      reinterpret_cast<__nv_bfloat16*>(out)[e] = __float2bfloat16_rn(acc);
+    else
+      reinterpret_cast<float*>(out)[e] = acc;
+  }
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+__global__ void swiglu_fwd_kernel(const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ u,
+                                  __nv_bfloat16* __restrict__ h, long long numel) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < numel; e += stride) {
+    const float gv = __bfloat162float(g[e]);
+    const float uv = __bfloat162float(u[e]);
+    h[e] = __float2bfloat16_rn(silu_f(gv) * uv);
+  }
+}
+
+__global__ void swiglu_bwd_kernel(const __nv_bfloat16* dh, const __nv_bfloat16* __restrict__ g,
+                                  const __nv_bfloat16* __restrict__ u, __nv_bfloat16* dg, __nv_bfloat16* du,
+                                  long long numel) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < numel; e += stride) {
+    const float gv = __bfloat162float(g[e]);
+    const float uv = __bfloat162float(u[e]);
+    const float dv = __bfloat162float(dh[e]);
+    const float sg = 1.0f / (1.0f + expf(-gv));
+    const float silu = gv * sg;
+    const float dsilu = sg * (1.0f + gv * (1.0f - sg));
+    dg[e] = __float2bfloat16_rn(dv * uv * dsilu);
+    du[e] = __float2bfloat16_rn(dv * silu);
+  }
+}
+
+// Waits on a barrier that expects one arrival nobody makes; the bounded wait must give up and latch the
+// timeout bit.  Used only by ql_selftest_wait_timeout.
+__global__ void selftest_wait_kernel(long long limit, unsigned int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err, limit);
+  __syncthreads();
+}
+
+}  // namespace qlora

@@ -1,0 +1,284 @@
+"""Python binding of libqlora (the C ABI in include/qlora.h): argument marshalling only.
+
+Every function here allocates its outputs with PyTorch on the inputs' CUDA device, passes raw pointers
+and the current CUDA stream to the library, and raises ``QLoRAError`` on a non-OK status.  All arithmetic
+runs in the library's kernels; there is no fallback: if libqlora.so is missing, the first call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora.so")
+
+QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_CUDA, QL_ERR_TIMEOUT = range(5)
+QL_F32, QL_BF16 = 0, 1
+QL_PASS_FWD, QL_PASS_BWD = 0, 1
+
+_lib = None
+_lock = threading.Lock()
+
+_c_i64 = ctypes.c_int64
+_c_p = ctypes.c_void_p
+
+# name -> (restype, argtypes): mirrors include/qlora.h
+SIGNATURES = {
+    "ql_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ql_abi_version": (ctypes.c_int, []),
+    "ql_nf4_codebook": (None, [ctypes.POINTER(ctypes.c_float)]),
+    "ql_get_device_error": (ctypes.c_int, [_c_p]),
+    "ql_launch_count": (ctypes.c_uint64, []),
+    "ql_set_profile_events": (ctypes.c_int, [ctypes.c_int, _c_p, _c_p]),
+    "ql_selftest_wait_timeout": (ctypes.c_int, [_c_i64, _c_p]),
+    "nf4_quantize": (ctypes.c_int, [_c_p, _c_i64, ctypes.c_int, _c_p, _c_p, _c_p]),
+    "nf4_dequantize": (ctypes.c_int, [_c_p, _c_p, _c_i64, ctypes.c_int, ctypes.c_int, _c_p, _c_p]),
+    "qlora_workspace_bytes": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64, _c_i64, ctypes.c_int]),
+    "qlora_linear_fwd": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, ctypes.c_float,
+                                        _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
+    "qlora_linear_bwd": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                        ctypes.c_float, _c_p, _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
+    "qlora_swiglu_fwd": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, _c_p]),
+    "qlora_swiglu_bwd": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+}
+
+
+class QLoRAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(f"libqlora.so is not built ({LIB_PATH}); run "
+                                       "`python -m qlora_fine_tuning_blockwise_b200.build`")
+                L = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in SIGNATURES.items():
+                    f = getattr(L, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().ql_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != QL_OK:
+        raise QLoRAError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device | None = None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    """bf16 tensors travel as their bit patterns; the library reads them as uint16."""
+    assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous(), (t.dtype, t.device, t.is_contiguous())
+    return t
+
+
+# ------------------------------------------------------------------------------------------ host-only
+
+
+def abi_version() -> int:
+    return int(lib().ql_abi_version())
+
+
+def codebook() -> np.ndarray:
+    """The library's NF4 table (fp32, ascending)."""
+    out = (ctypes.c_float * 16)()
+    lib().ql_nf4_codebook(out)
+    return np.array(out[:], dtype=np.float32)
+
+
+def workspace_bytes(M: int, N: int, K: int, r: int, pass_: int) -> int:
+    return int(lib().qlora_workspace_bytes(M, N, K, r, pass_))
+
+
+def device_error(device: torch.device | None = None) -> int:
+    """Status from the device error word (synchronizes the current stream)."""
+    return int(lib().ql_get_device_error(_stream(device)))
+
+
+def launch_count() -> int:
+    """Kernels this library has launched in this process."""
+    return int(lib().ql_launch_count())
+
+
+def set_profile_events(which: int, start=None, stop=None) -> None:
+    """Record torch.cuda.Event ``start``/``stop`` around the fused forward (0) or dX (1) GEMM; None disables."""
+    def handle(ev):
+        if ev is None:
+            return None
+        if ev.cuda_event == 0:  # torch creates the event on first record
+            ev.record()
+        return ctypes.c_void_p(ev.cuda_event)
+    _check(lib().ql_set_profile_events(which, handle(start), handle(stop)), "ql_set_profile_events")
+
+
+def selftest_wait_timeout(wait_cycles: int) -> None:
+    _check(lib().ql_selftest_wait_timeout(int(wait_cycles), _stream()), "ql_selftest_wait_timeout")
+
+
+# ------------------------------------------------------------------------------------------ NF4
+
+
+def nf4_quantize(w: torch.Tensor, blocksize: int = 64):
+    """w: CUDA fp32 (any shape, row-major contiguous) -> (codes uint8 [numel/2], absmax fp32 [numel/blocksize])."""
+    assert w.is_cuda and w.dtype == torch.float32 and w.is_contiguous()
+    n = w.numel()
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=w.device)
+    absmax = torch.empty(max(n // max(blocksize, 1), 0), dtype=torch.float32, device=w.device)
+    _check(lib().nf4_quantize(_ptr(w), n, blocksize, _ptr(codes), _ptr(absmax), _stream(w.device)), "nf4_quantize")
+    return codes, absmax
+
+
+def nf4_dequantize(codes: torch.Tensor, absmax: torch.Tensor, numel: int, blocksize: int = 64,
+                   dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    assert codes.is_cuda and codes.dtype == torch.uint8 and absmax.dtype == torch.float32
+    out = torch.empty(numel, dtype=dtype, device=codes.device)
+    code = QL_BF16 if dtype == torch.bfloat16 else QL_F32
+    _check(lib().nf4_dequantize(_ptr(codes), _ptr(absmax), numel, blocksize, code, _ptr(out), _stream(codes.device)),
+           "nf4_dequantize")
+    return out
+
+
+# ------------------------------------------------------------------------------------------ linear layer
+
+
+def _workspace(M, N, K, r, pass_, device, workspace):
+    need = workspace_bytes(M, N, K, r, pass_)
+    if workspace is not None and workspace.numel() >= need:
+        return workspace, need
+    return (torch.empty(need, dtype=torch.uint8, device=device) if need else None), need
+
+
+def qlora_linear_fwd(x, codes, absmax, A, B, s: float, N: int, K: int, want_su: bool = True, workspace=None,
+                     y=None, su=None):
+    """(y [M,N] bf16, su [M,r] bf16 or None) for y = x deq(W)^T + s (x A^T) B^T."""
+    M = x.shape[0]
+    r = 0 if A is None else A.shape[0]
+    dev = x.device
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if y is None else y
+    if want_su and r > 0 and su is None:
+        su = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    if not want_su:
+        su = None
+    ws, need = _workspace(M, N, K, r, QL_PASS_FWD, dev, workspace)
+    _check(lib().qlora_linear_fwd(M, N, K, r, _ptr(_bits(x)), _ptr(codes), _ptr(absmax),
+                                  _ptr(A if r else None), _ptr(B if r else None), float(s), _ptr(y), _ptr(su),
+                                  _ptr(ws), need, _stream(dev)), "qlora_linear_fwd")
+    return y, su
+
+
+def qlora_linear_bwd(dy, x, codes, absmax, A, B, s: float, N: int, K: int, su=None, need_dx=True, need_dA=True,
+                     need_dB=True, workspace=None, dx=None, dA=None, dB=None):
+    """(dX [M,K] bf16, dA [r,K] fp32, dB [N,r] fp32); entries not requested are None."""
+    M = dy.shape[0]
+    r = 0 if A is None else A.shape[0]
+    dev = dy.device
+    if need_dx and dx is None:
+        dx = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    if need_dA and r > 0 and dA is None:
+        dA = torch.empty(r, K, dtype=torch.float32, device=dev)
+    if need_dB and r > 0 and dB is None:
+        dB = torch.empty(N, r, dtype=torch.float32, device=dev)
+    dx = dx if need_dx else None
+    dA = dA if (need_dA and r > 0) else None
+    dB = dB if (need_dB and r > 0) else None
+    ws, need = _workspace(M, N, K, r, QL_PASS_BWD, dev, workspace)
+    _check(lib().qlora_linear_bwd(M, N, K, r, _ptr(dy), _ptr(x), _ptr(codes), _ptr(absmax),
+                                  _ptr(A if r else None), _ptr(B if r else None), float(s), _ptr(su), _ptr(dx),
+                                  _ptr(dA), _ptr(dB), _ptr(ws), need, _stream(dev)), "qlora_linear_bwd")
+    return dx, dA, dB
+
+
+# ------------------------------------------------------------------------------------------ SwiGLU
+
+
+def swiglu_fwd(g: torch.Tensor, u: torch.Tensor, h: torch.Tensor | None = None) -> torch.Tensor:
+    h = torch.empty_like(g) if h is None else h
+    _check(lib().qlora_swiglu_fwd(g.numel(), _ptr(_bits(g)), _ptr(_bits(u)), _ptr(h), _stream(g.device)),
+           "qlora_swiglu_fwd")
+    return h
+
+
+def swiglu_bwd(dh: torch.Tensor, g: torch.Tensor, u: torch.Tensor, dg=None, du=None):
+    dg = torch.empty_like(g) if dg is None else dg
+    du = torch.empty_like(u) if du is None else du
+    _check(lib().qlora_swiglu_bwd(g.numel(), _ptr(_bits(dh)), _ptr(g), _ptr(u), _ptr(dg), _ptr(du),
+                                  _stream(g.device)), "qlora_swiglu_bwd")
+    return dg, du
+
+
+# ------------------------------------------------------------------------------------------ a layer object
+
+
+class QLoRALinear:
+    """A frozen NF4 base weight with its bf16 LoRA pair and preallocated buffers for repeated steps.
+
+    ``forward`` / ``backward`` reuse the output and workspace buffers of the last call with the same M, so a
+    training loop allocates nothing per step.
+    """
+
+    def __init__(self, W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, s: float):
+        assert W.dim() == 2 and W.is_cuda
+        self.N, self.K = W.shape
+        self.codes, self.absmax = nf4_quantize(W.contiguous())
+        self.A, self.B, self.s = A, B, float(s)
+        self.r = 0 if A is None else A.shape[0]
+        self._bufs = {}
+
+    @classmethod
+    def from_quantized(cls, codes, absmax, N, K, A, B, s):
+        self = cls.__new__(cls)
+        self.N, self.K = N, K
+        self.codes, self.absmax = codes, absmax
+        self.A, self.B, self.s = A, B, float(s)
+        self.r = 0 if A is None else A.shape[0]
+        self._bufs = {}
+        return self
+
+    def _buffers(self, M: int, device):
+        b = self._bufs.get(M)
+        if b is None:
+            N, K, r = self.N, self.K, self.r
+            b = dict(
+                y=torch.empty(M, N, dtype=torch.bfloat16, device=device),
+                su=torch.empty(M, r, dtype=torch.bfloat16, device=device) if r else None,
+                dx=torch.empty(M, K, dtype=torch.bfloat16, device=device),
+                dA=torch.empty(r, K, dtype=torch.float32, device=device) if r else None,
+                dB=torch.empty(N, r, dtype=torch.float32, device=device) if r else None,
+                ws_f=torch.empty(max(workspace_bytes(M, N, K, r, QL_PASS_FWD), 1), dtype=torch.uint8, device=device),
+                ws_b=torch.empty(max(workspace_bytes(M, N, K, r, QL_PASS_BWD), 1), dtype=torch.uint8, device=device),
+            )
+            self._bufs[M] = b
+        return b
+
+    def forward(self, x: torch.Tensor):
+        b = self._buffers(x.shape[0], x.device)
+        return qlora_linear_fwd(x, self.codes, self.absmax, self.A, self.B, self.s, self.N, self.K, want_su=True,
+                                workspace=b["ws_f"], y=b["y"], su=b["su"])
+
+    def backward(self, dy: torch.Tensor, x: torch.Tensor, su: torch.Tensor | None = None, need_dx: bool = True):
+        b = self._buffers(dy.shape[0], dy.device)
+        return qlora_linear_bwd(dy, x, self.codes, self.absmax, self.A, self.B, self.s, self.N, self.K, su=su,
+                                need_dx=need_dx, workspace=b["ws_b"], dx=b["dx"], dA=b["dA"], dB=b["dB"])

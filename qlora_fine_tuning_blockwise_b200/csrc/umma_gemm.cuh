@@ -10,14 +10,15 @@
 //
 // Operand A, per stage (128 rows x 64 contraction elements, bf16, 128-byte swizzled canonical layout):
 //   A_TMA_K / A_TMA_MN   loaded by TMA from a bf16 matrix (K-major or MN-major),
-//   A_DEQ_K              dequantized from NF4 codes by 8 producer warps (forward: rows = W rows n, K-major),
+//   A_DEQ_K              dequantized from NF4 codes by producer warps (forward: rows = W rows n, K-major),
 //   A_DEQ_MN             dequantized the same way into the MN-major layout (backward: rows = W columns k,
 //                        contraction over W rows n) -- the transpose of deq(W) costs nothing extra.
 //   The codes arrive by TMA into a shared-memory ring; absmax is read with __ldg one stage ahead.
 // Operand B (BN x 64): always by TMA (K-major or MN-major).
 //
 // Warp roles: warp 0 = TMA producer (one thread), warp 1 = TMEM allocator + MMA issuer (one thread),
-// warps 2..9 = dequantizers (A_DEQ_* only), warps 2..5 = epilogue (TMEM -> registers -> global).
+// warps 2..9 = dequantizers (A_DEQ_* only, two groups of 4 alternating over stages), warps 2..5 = epilogue
+// (TMEM -> registers -> global).
 //
 // Shared-memory tiles: for the 128B swizzle every tile starts on a 1024-byte boundary; row r of a tile is
 // 128 bytes at r*128 and its 16-byte chunk c sits at chunk position c ^ (r & 7).  TMA writes that layout;
@@ -58,14 +59,15 @@ struct UmmaCfg {
   static constexpr int kBBytes = BN * 64 * 2;
   static constexpr int kCBytes = kDeq ? 4096 : 0;
   static constexpr int kStageBytes = kABytes + kBBytes + kCBytes;
-  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kLutBytes = kDeq ? 256 * 8 : 0;
-  static constexpr int kDeqWarps = kDeq ? 8 : 0;
+  static constexpr int kStagesRaw = (210 * 1024) / kStageBytes;
+  static constexpr int kStagesCap = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // the two dequantizer groups alternate over main stages; with an even ring every slot keeps one group
+  static constexpr int kStages = kDeq ? (kStagesCap & ~1) : kStagesCap;
+  static constexpr int kDeqWarpsPerGroup = 4;
   static constexpr int kThreads = 64 + (kDeq ? 256 : 128);
   static constexpr int kTmemCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
   static constexpr int kBarBytes = 512;  // 4 barrier arrays x 8 stages + accumulator barrier + TMEM slot + abort flag
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kLutBytes + kBarBytes;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is a multiple of 16 in [16, 256]");
   static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-element swizzle atoms");
   static_assert(kStages >= 2, "pipeline needs two stages");
@@ -73,11 +75,55 @@ struct UmmaCfg {
   static_assert((4 * kStages + 1) * 8 + 8 <= kBarBytes, "barrier area");
 };
 
-// Dequantize one byte (two codes, high nibble first) into a bf16 pair: low half = first element.
-__device__ __forceinline__ uint32_t deq_pair(const float2* lut, uint32_t byte, float sc) {
-  const float2 l = lut[byte];
-  __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(l.x, sc), __fmul_rn(l.y, sc));
-  return *reinterpret_cast<uint32_t*>(&h);
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// The 16 levels of one block scaled by its absmax and rounded to bf16 -- exactly the values
+// nf4_dequantize(..., bf16) produces -- held in registers as byte planes for byte-permute lookups:
+// lo[j] holds the low bytes of entries 4j..4j+3, hi[j] their high bytes.
+struct Nf4RegTable {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ Nf4RegTable nf4_reg_table(float sc) {
+  const float lv[16] = {QLORA_NF4_LEVELS};
+  uint32_t p[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(lv[2 * i], sc), __fmul_rn(lv[2 * i + 1], sc));
+    p[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  Nf4RegTable t;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    t.lo[j] = prmt(p[2 * j], p[2 * j + 1], 0x6420u);
+    t.hi[j] = prmt(p[2 * j], p[2 * j + 1], 0x7531u);
+  }
+  return t;
+}
+
+// Eight codes (one 32-bit word: byte j = element 2j in the high nibble, 2j+1 in the low nibble) ->
+// eight bf16 values in element order (four bf16 pairs, first element in the low half).
+// Each nibble v selects byte (v & 7) of the table half v >> 3; a byte mask from bit 3 picks the half.
+__device__ __forceinline__ void nf4_lookup8(const Nf4RegTable& t, uint32_t q, uint32_t (&o)[4]) {
+  const uint32_t s0 = q & 0x77777777u;
+  const uint32_t b0 = (q >> 3) & 0x11111111u;
+  const uint32_t s1 = s0 >> 16;
+  const uint32_t b1 = b0 >> 16;
+  const uint32_t m0 = prmt(0x0000FF00u, 0u, b0);  // byte i: 0xFF when code (i ^ 1) of the low half is >= 8
+  const uint32_t m1 = prmt(0x0000FF00u, 0u, b1);
+  const uint32_t L0 = (prmt(t.lo[0], t.lo[1], s0) & ~m0) | (prmt(t.lo[2], t.lo[3], s0) & m0);
+  const uint32_t H0 = (prmt(t.hi[0], t.hi[1], s0) & ~m0) | (prmt(t.hi[2], t.hi[3], s0) & m0);
+  const uint32_t L1 = (prmt(t.lo[0], t.lo[1], s1) & ~m1) | (prmt(t.lo[2], t.lo[3], s1) & m1);
+  const uint32_t H1 = (prmt(t.hi[0], t.hi[1], s1) & ~m1) | (prmt(t.hi[2], t.hi[3], s1) & m1);
+  // L0/H0 hold elements in the order (1, 0, 3, 2); interleave low and high bytes back into element order
+  o[0] = prmt(L0, H0, 0x4051u);
+  o[1] = prmt(L0, H0, 0x6273u);
+  o[2] = prmt(L1, H1, 0x4051u);
+  o[3] = prmt(L1, H1, 0x6273u);
 }
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, unsigned int* err) {
@@ -104,11 +150,10 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = sA + ST * C::kABytes;
   uint8_t* sC = sB + ST * C::kBBytes;
-  float2* lut = reinterpret_cast<float2*>(sC + ST * C::kCBytes);
   // Barrier phases: full_tma[s] and empty[s] advance once per use of slot s (every stage); full_codes[s]
   // and full_deq[s] once per MAIN-stage use of slot s (the LoRA stages carry no codes).  Each waiter visits
   // every phase of the barriers it waits on, so a parity wait never aliases an older phase.
-  uint64_t* full_tma = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(lut) + C::kLutBytes);
+  uint64_t* full_tma = reinterpret_cast<uint64_t*>(sC + ST * C::kCBytes);
   uint64_t* full_codes = full_tma + ST;
   uint64_t* full_deq = full_codes + ST;
   uint64_t* empty = full_deq + ST;
@@ -133,15 +178,12 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full_tma[s], 1);
       mbar_init(&full_codes[s], 1);
-      mbar_init(&full_deq[s], C::kDeqWarps > 0 ? C::kDeqWarps : 1);
+      mbar_init(&full_deq[s], C::kDeqWarpsPerGroup);
       mbar_init(&empty[s], 1);
     }
     mbar_init(accum_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
-  }
-  if constexpr (C::kDeq) {
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) lut[b] = make_float2(kNF4LevelsDev[b >> 4], kNF4LevelsDev[b & 15]);
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmB);
@@ -248,55 +290,45 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
   } else {
     // ------------------------------------------------------------------ dequantizers (warps 2..9)
     if constexpr (C::kDeq) {
+      // Two groups of 4 warps take alternate main stages; a thread expands one 64-element block row:
+      //   A_DEQ_K : thread = W row n of the stage (128 rows x 64 k), K-major tile,
+      //   A_DEQ_MN: thread = (W row n of the stage, half h of the 128-wide k range), MN-major tile;
+      //             rows map so that the 8 lanes of a store phase hit 8 distinct 16-byte bank groups.
       const int t = threadIdx.x - 64;  // 0..255
-      // A_DEQ_K : row = W row n (0..127), half selects k 0..31 / 32..63 of the stage
-      // A_DEQ_MN: row = W row n (0..63) of the stage, q selects k 32q..32q+31 of the 128-wide tile
-      const int row = (AM == A_DEQ_K) ? (t >> 1) : (t >> 2);
-      const int sub = (AM == A_DEQ_K) ? (t & 1) : (t & 3);
-      const int c_off = (AM == A_DEQ_K) ? (row * 32 + sub * 16) : (row * 64 + sub * 16);
+      const int grp = t >> 7;
+      const int tg = t & 127;
+      const int row = (AM == A_DEQ_K) ? tg : ((tg & 7) + 8 * (tg >> 4));
+      const int h = (AM == A_DEQ_K) ? 0 : ((tg >> 3) & 1);
+      const int c_off = (AM == A_DEQ_K) ? row * 32 : (row * 64 + h * 32);
+      const int a_off = (AM == A_DEQ_K) ? row * 128 : (h * 8192 + row * 128);
 
       auto scale_of = [&](int it) -> float {
         const int kk0 = (main_begin + it - n_extra) * 64;
-        int n, k;
-        if (AM == A_DEQ_K) {
-          n = i0 + row;
-          k = kk0;
-        } else {
-          n = kk0 + row;
-          k = i0 + sub * 32;
-        }
+        const int n = (AM == A_DEQ_K) ? (i0 + row) : (kk0 + row);
+        const int k = (AM == A_DEQ_K) ? kk0 : (i0 + 64 * h);
         if (n < args.w_rows && k < args.w_cols) return __ldg(args.absmax + static_cast<long long>(n) * args.w_kb + (k >> 6));
         return 0.0f;
       };
 
-      float sc_next = (n_extra < n_total) ? scale_of(n_extra) : 0.0f;
-      uint32_t codes_phase = 0;  // bit s: parity of the next full_codes[s] phase (main-stage uses of slot s)
-      for (int it = n_extra; it < n_total; ++it) {
+      const int first = n_extra + grp;
+      float sc_next = (first < n_total) ? scale_of(first) : 0.0f;
+      uint32_t codes_phase = 0;  // bit s: parity of the next full_codes[s] phase this group waits for
+      for (int it = first; it < n_total; it += 2) {
         const int s = it % ST;
         const float sc = sc_next;
-        if (it + 1 < n_total) sc_next = scale_of(it + 1);
+        if (it + 2 < n_total) sc_next = scale_of(it + 2);
+        const Nf4RegTable tab = nf4_reg_table(sc);
         if (!mbar_wait(&full_codes[s], (codes_phase >> s) & 1u, abort_flag, args.err)) break;
         codes_phase ^= 1u << s;
-        const uint4 cw = *reinterpret_cast<const uint4*>(sC + s * C::kCBytes + c_off);
-        uint8_t* a_tile = sA + s * C::kABytes;
-        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        const uint4 c01 = *reinterpret_cast<const uint4*>(sC + s * C::kCBytes + c_off);
+        const uint4 c23 = *reinterpret_cast<const uint4*>(sC + s * C::kCBytes + c_off + 16);
+        const uint32_t words[8] = {c01.x, c01.y, c01.z, c01.w, c23.x, c23.y, c23.z, c23.w};
+        uint8_t* a_row = sA + s * C::kABytes + a_off;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const uint32_t w = words[p];
-          uint4 o;
-          o.x = deq_pair(lut, w & 0xFFu, sc);
-          o.y = deq_pair(lut, (w >> 8) & 0xFFu, sc);
-          o.z = deq_pair(lut, (w >> 16) & 0xFFu, sc);
-          o.w = deq_pair(lut, w >> 24, sc);
-          uint8_t* dst;
-          if (AM == A_DEQ_K) {
-            const int chunk = sub * 4 + p;
-            dst = a_tile + row * 128 + ((chunk ^ (row & 7)) << 4);
-          } else {
-            const int chunk = ((sub & 1) << 2) | p;
-            dst = a_tile + (sub >> 1) * 8192 + row * 128 + ((chunk ^ (row & 7)) << 4);
-          }
-          *reinterpret_cast<uint4*>(dst) = o;
+        for (int w = 0; w < 8; ++w) {
+          uint32_t o[4];
+          nf4_lookup8(tab, words[w], o);
+          *reinterpret_cast<uint4*>(a_row + ((w ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();

@@ -138,6 +138,24 @@ QL_API ql_status qlora_linear_fwd(int64_t M, int64_t N, int64_t K, int64_t r, co
                            uint16_t* su_out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * qlora_linear_fwd_noalloc -- the forward above for callers that cannot allocate device memory at all, not
+ * even a workspace to lend: code running while a stream is captured in global mode (where cudaMalloc is an
+ * error) or a plug-in whose host program owns all device memory and forbids allocation after start-up.
+ * The paper has no counterpart; this is a property of this library's interface.
+ *   Arguments as qlora_linear_fwd, without workspace/ws_bytes.  The scratch lives in an 8 MiB array
+ *   compiled into the library, which every GPU that loads the library holds until the process exits.
+ *   Sizes whose qlora_workspace_bytes(M,N,K,r,QL_PASS_FWD) exceeds 8 MiB (8388608 bytes) return
+ *   QL_ERR_INVALID_ARG before any launch.  No cudaMalloc, cudaFree or allocating routine is called.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that device
+ *   current; make that first call before any stream capture.  All calls share the one array and it keeps
+ *   the last call's contents (the forward overwrites every scratch byte it reads), so calls that overlap on
+ *   the GPU -- on different streams, or from several threads -- race; serialize them.
+ */
+QL_API ql_status qlora_linear_fwd_noalloc(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x,
+                                          const uint8_t* codes, const float* absmax, const uint16_t* A,
+                                          const uint16_t* B, float s, uint16_t* y, uint16_t* su_out, void* stream);
+
+/*
  * qlora_linear_bwd -- gradients of the layer with the base weight frozen ("How LoRA and QLoRA work": only
  * the adapters train; "Unsloth v0.1.47-beta ..." (kongchang.com), section on LoRA/QLoRA: the rewritten
  * backward keeps numerical equivalence).

@@ -621,3 +621,50 @@ ql_status qlora_swiglu_bwd(int64_t numel, const uint16_t* dh, const uint16_t* g,
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------ no-allocation forward
+//
+// Some callers cannot allocate device memory at all, not even a workspace to lend the library: code that
+// runs while a stream is being captured in global mode (where cudaMalloc is an error), or a plug-in hosted
+// by a program that owns all device memory and forbids allocations once it has started.  For them
+// qlora_linear_fwd_noalloc runs the forward with its scratch in a fixed array compiled into the library.
+
+namespace qlora {
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB on every device that loads the library
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+// Device address of g_noalloc_scratch per device.  In host code the array's name is only a host-side
+// stand-in, so the address is looked up once per device, with that device current.
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+bool noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return false;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return true;
+}
+
+}  // namespace
+}  // namespace qlora
+
+extern "C" ql_status qlora_linear_fwd_noalloc(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x,
+                                              const uint8_t* codes, const float* absmax, const uint16_t* A,
+                                              const uint16_t* B, float s, uint16_t* y, uint16_t* su_out,
+                                              void* stream) {
+  const ql_status st = check_linear(M, N, K, r);
+  if (st != QL_OK) return st;
+  if (qlora_workspace_bytes(M, N, K, r, QL_PASS_FWD) > kNoallocScratchBytes) return QL_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if (!noalloc_scratch(&scratch)) return QL_ERR_CUDA;
+  return qlora_linear_fwd(M, N, K, r, x, codes, absmax, A, B, s, y, su_out, scratch, kNoallocScratchBytes, stream);
+}

@@ -43,6 +43,8 @@ SIGNATURES = {
                                         _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
     "qlora_linear_bwd": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
                                         ctypes.c_float, _c_p, _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
+    "qlora_linear_fwd_noalloc": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                                ctypes.c_float, _c_p, _c_p, _c_p]),
     "qlora_swiglu_fwd": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, _c_p]),
     "qlora_swiglu_bwd": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
 }
@@ -186,6 +188,17 @@ def qlora_linear_fwd(x, codes, absmax, A, B, s: float, N: int, K: int, want_su: 
     _check(lib().qlora_linear_fwd(M, N, K, r, _ptr(_bits(x)), _ptr(codes), _ptr(absmax),
                                   _ptr(A if r else None), _ptr(B if r else None), float(s), _ptr(y), _ptr(su),
                                   _ptr(ws), need, _stream(dev)), "qlora_linear_fwd")
+    return y, su
+
+
+def qlora_linear_fwd_noalloc(x, codes, absmax, A, B, s: float, N: int, K: int, y, su=None):
+    """The forward with the library's built-in scratch instead of a workspace (for callers that cannot
+    allocate device memory); ``y`` (and ``su`` when wanted) are the caller's buffers.  Returns (y, su)."""
+    M = x.shape[0]
+    r = 0 if A is None else A.shape[0]
+    _check(lib().qlora_linear_fwd_noalloc(M, N, K, r, _ptr(_bits(x)), _ptr(codes), _ptr(absmax),
+                                          _ptr(A if r else None), _ptr(B if r else None), float(s), _ptr(y),
+                                          _ptr(su), _stream(x.device)), "qlora_linear_fwd_noalloc")
     return y, su
 
 

@@ -178,6 +178,7 @@ def run_ours(args, rank, world, local, peaks):
     from qlora_fine_tuning_blockwise_b200 import build as qbuild
     from qlora_fine_tuning_blockwise_b200 import inputs as I
     from qlora_fine_tuning_blockwise_b200 import ops
+    from qlora_fine_tuning_blockwise_b200.parallel import allreduce_adapter_grads
 
     qbuild.build()
     w = I.WORKLOADS[args.workload]
@@ -197,8 +198,7 @@ def run_ours(args, rank, world, local, peaks):
         y, su = layer.forward(x)
         dx, dA, dB = layer.backward(dy, x, su=su)
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            allreduce_adapter_grads([dA, dB])
         return y, dx, dA, dB
 
     for _ in range(args.warmup):
@@ -273,6 +273,8 @@ def run_e2e(ctx, args, world):
     import torch
     import torch.distributed as dist
 
+    from qlora_fine_tuning_blockwise_b200.parallel import allreduce_adapter_grads
+
     layer, x_dev, dy_dev, d, w, dev = ctx
     x_h = d["x"].pin_memory()
     dy_h = d["dy"].pin_memory()
@@ -287,8 +289,7 @@ def run_e2e(ctx, args, world):
         y, su = layer.forward(x)
         dx, dA, dB = layer.backward(dy, x, su=su)
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            allreduce_adapter_grads([dA, dB])
         if outs_h is None:
             outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (y, dx, dA, dB)]
         for h, t in zip(outs_h, (y, dx, dA, dB)):

@@ -189,6 +189,22 @@ QL_API ql_status qlora_swiglu_fwd(int64_t numel, const uint16_t* g, const uint16
 QL_API ql_status qlora_swiglu_bwd(int64_t numel, const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,
                            uint16_t* du, void* stream);
 
+/*
+ * qlora_swiglu_gated_fwd -- SwiGLU over the output of the fused gate/up projection of a gated MLP
+ * ("Inside Unsloth ...", section "What You'll Learn", item "Triton Kernel Internals": the SwiGLU kernels).
+ * gu is bf16 [M, 2F]: row m holds the gate pre-activation g in columns [0, F) and the up projection in
+ * [F, 2F) -- the y of qlora_linear_fwd on the stacked weight [W_gate; W_up].  h = silu(g) * up, bf16
+ * [M, F], computed in fp32.  F % 8 == 0; buffers 16-byte aligned.
+ */
+QL_API ql_status qlora_swiglu_gated_fwd(int64_t M, int64_t F, const uint16_t* gu, uint16_t* h, void* stream);
+
+/*
+ * qlora_swiglu_gated_bwd -- its backward: dgu [M, 2F] bf16 receives dh * up * silu'(g) in columns [0, F)
+ * and dh * silu(g) in [F, 2F): the upstream gradient of the stacked gate/up projection.  dh bf16 [M, F].
+ */
+QL_API ql_status qlora_swiglu_gated_bwd(int64_t M, int64_t F, const uint16_t* dh, const uint16_t* gu,
+                                        uint16_t* dgu, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -620,6 +620,32 @@ ql_status qlora_swiglu_bwd(int64_t numel, const uint16_t* dh, const uint16_t* g,
   return status_of(cudaGetLastError());
 }
 
+ql_status qlora_swiglu_gated_fwd(int64_t M, int64_t F, const uint16_t* gu, uint16_t* h, void* stream) {
+  if (M < 0 || F < 0 || F % 8 != 0) return QL_ERR_INVALID_ARG;
+  if (M == 0 || F == 0) return QL_OK;
+  if (!gu || !h || !aligned16(gu) || !aligned16(h)) return QL_ERR_INVALID_ARG;
+  const int threads = 256;
+  const long long ctas = std::min<long long>(cdiv(M * (F / 8), threads), 148LL * 32);
+  swiglu_gated_fwd_kernel<<<static_cast<unsigned>(ctas), threads, 0, as_stream(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(gu), reinterpret_cast<__nv_bfloat16*>(h), M, F);
+  count_launch();
+  return status_of(cudaGetLastError());
+}
+
+ql_status qlora_swiglu_gated_bwd(int64_t M, int64_t F, const uint16_t* dh, const uint16_t* gu, uint16_t* dgu,
+                                 void* stream) {
+  if (M < 0 || F < 0 || F % 8 != 0) return QL_ERR_INVALID_ARG;
+  if (M == 0 || F == 0) return QL_OK;
+  if (!dh || !gu || !dgu || !aligned16(dh) || !aligned16(gu) || !aligned16(dgu)) return QL_ERR_INVALID_ARG;
+  const int threads = 256;
+  const long long ctas = std::min<long long>(cdiv(M * (F / 8), threads), 148LL * 32);
+  swiglu_gated_bwd_kernel<<<static_cast<unsigned>(ctas), threads, 0, as_stream(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(dh), reinterpret_cast<const __nv_bfloat16*>(gu),
+      reinterpret_cast<__nv_bfloat16*>(dgu), M, F);
+  count_launch();
+  return status_of(cudaGetLastError());
+}
+
 }  // extern "C"
 
 // ------------------------------------------------------------------------------------------ no-allocation forward

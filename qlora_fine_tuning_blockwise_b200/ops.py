@@ -47,6 +47,8 @@ SIGNATURES = {
                                                 ctypes.c_float, _c_p, _c_p, _c_p]),
     "qlora_swiglu_fwd": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, _c_p]),
     "qlora_swiglu_bwd": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    "qlora_swiglu_gated_fwd": (ctypes.c_int, [_c_i64, _c_i64, _c_p, _c_p, _c_p]),
+    "qlora_swiglu_gated_bwd": (ctypes.c_int, [_c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
 }
 
 
@@ -240,6 +242,24 @@ def swiglu_bwd(dh: torch.Tensor, g: torch.Tensor, u: torch.Tensor, dg=None, du=N
     _check(lib().qlora_swiglu_bwd(g.numel(), _ptr(_bits(dh)), _ptr(g), _ptr(u), _ptr(dg), _ptr(du),
                                   _stream(g.device)), "qlora_swiglu_bwd")
     return dg, du
+
+
+def swiglu_gated_fwd(gu: torch.Tensor, h: torch.Tensor | None = None) -> torch.Tensor:
+    """gu bf16 [M, 2F] (gate | up) -> h bf16 [M, F]."""
+    M, F2 = gu.shape
+    h = torch.empty(M, F2 // 2, dtype=torch.bfloat16, device=gu.device) if h is None else h
+    _check(lib().qlora_swiglu_gated_fwd(M, F2 // 2, _ptr(_bits(gu)), _ptr(h), _stream(gu.device)),
+           "qlora_swiglu_gated_fwd")
+    return h
+
+
+def swiglu_gated_bwd(dh: torch.Tensor, gu: torch.Tensor, dgu: torch.Tensor | None = None) -> torch.Tensor:
+    """(dh [M, F], gu [M, 2F]) -> dgu [M, 2F] bf16."""
+    M, F2 = gu.shape
+    dgu = torch.empty_like(gu) if dgu is None else dgu
+    _check(lib().qlora_swiglu_gated_bwd(M, F2 // 2, _ptr(_bits(dh)), _ptr(gu), _ptr(dgu), _stream(gu.device)),
+           "qlora_swiglu_gated_bwd")
+    return dgu
 
 
 # ------------------------------------------------------------------------------------------ a layer object

@@ -132,6 +132,7 @@ struct GemmCall {
   int n_extra = 0;
   int splits = 1;
   int prof = -1;          // profiling-event slot recorded around this launch (-1: none)
+  int ctas = 148;         // persistent CTAs: at most one per SM
   UmmaArgs args{};
 };
 
@@ -162,7 +163,7 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
   }
   if (C::kDeq) {
     const int64_t N = g.args.w_rows, K = g.args.w_cols;
-    if (AM == A_DEQ_K) {
+    if (AM == A_DEQ_K || AM == A_DEQ_TMEM) {
       if (!make_map(&tmC, g.codes, N, K / 2, 1, 32, 128, false)) return cudaErrorInvalidValue;
     } else {
       if (!make_map(&tmC, g.codes, N, K / 2, 1, 64, 64, false)) return cudaErrorInvalidValue;
@@ -171,8 +172,8 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
   auto kern = umma_gemm_kernel<BN, AM, BMN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(cdiv(g.cols, BN)), static_cast<unsigned>(cdiv(g.rows, 128)),
-            static_cast<unsigned>(g.splits));
+  const int64_t units = static_cast<int64_t>(g.args.splits) * g.args.tiles_i * g.args.tiles_j;
+  dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, g.ctas)));
   if (g.prof >= 0) prof_record(g.prof, 0, stream);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmBx, tmC, g.args);
   count_launch();
@@ -202,6 +203,7 @@ cudaError_t launch_bn(const GemmCall& g, cudaStream_t stream) {
 }
 
 cudaError_t launch_gemm(const GemmCall& g, cudaStream_t stream) {
+  if (g.am == A_DEQ_TMEM && !g.b_mn) return launch_bn<A_DEQ_TMEM, false>(g, stream);
   if (g.am == A_DEQ_K && !g.b_mn) return launch_bn<A_DEQ_K, false>(g, stream);
   if (g.am == A_DEQ_MN && !g.b_mn) return launch_bn<A_DEQ_MN, false>(g, stream);
   if (g.am == A_TMA_K && !g.b_mn) return launch_bn<A_TMA_K, false>(g, stream);
@@ -231,6 +233,23 @@ int plan_splits(int64_t tiles, int64_t kstages, int sms) {
   return s;
 }
 
+// Token-light layers (decode-like, at most 64 tokens) stream the weight once; split the contraction so the
+// persistent grid's makespan -- waves of units times stages per unit -- is smallest (at least 8 stages per
+// split, at most 8 splits: the fp32 partial sums cost extra traffic).
+int plan_splits_streaming(int64_t tiles, int64_t kstages, int sms) {
+  int best = 1;
+  int64_t best_cost = cdiv(tiles, sms) * kstages;
+  for (int s = 2; s <= 8; s *= 2) {
+    if (kstages < 8 * s) break;
+    const int64_t cost = cdiv(tiles * s, sms) * cdiv(kstages, s);
+    if (cost < best_cost) {
+      best = s;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 struct LinearPlan {
   int bn_main = 16, s_main = 1;      // forward y / backward dX
   int s_su = 1, s_v = 1, s_da = 1, s_db = 1;
@@ -242,13 +261,10 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass)
   LinearPlan p;
   const int sms = plan_sms();
   const int rp = rank_pad(r);
-  if (pass == QL_PASS_FWD) {
-    p.bn_main = main_bn(M);
-    p.s_main = plan_splits(cdiv(M, p.bn_main) * cdiv(N, 128), cdiv(K, 64), sms);
-  } else {
-    p.bn_main = main_bn(M);
-    p.s_main = plan_splits(cdiv(M, p.bn_main) * cdiv(K, 128), cdiv(N, 64), sms);
-  }
+  p.bn_main = main_bn(M);
+  const int64_t main_tiles = cdiv(M, p.bn_main) * (pass == QL_PASS_FWD ? cdiv(N, 128) : cdiv(K, 128));
+  const int64_t main_kst = pass == QL_PASS_FWD ? cdiv(K, 64) : cdiv(N, 64);
+  p.s_main = M <= 64 ? plan_splits_streaming(main_tiles, main_kst, sms) : plan_splits(main_tiles, main_kst, sms);
   size_t part = 0;
   if (p.s_main > 1) part = std::max(part, static_cast<size_t>(p.s_main) * M * (pass == QL_PASS_FWD ? N : K) * 4);
   if (r > 0) {
@@ -293,11 +309,15 @@ cudaError_t launch_reduce(const float* ws, int64_t slab, int nsplit, int64_t cou
 // `part` then one reduction.
 cudaError_t run_gemm(GemmCall g, void* out, bool out_bf16, float alpha, int64_t ls, int64_t cs, int64_t rows_lim,
                      int64_t cols_lim, int64_t count, float* part, unsigned int* err, cudaStream_t stream) {
+  g.ctas = plan_sms();
   g.args.rows = static_cast<int>(g.rows);
   g.args.cols = static_cast<int>(g.cols);
+  g.args.tiles_i = static_cast<int>(cdiv(g.rows, 128));
+  g.args.tiles_j = static_cast<int>(cdiv(g.cols, g.bn));
   g.args.k_stages = static_cast<int>(cdiv(g.k_total, 64));
   g.args.stages_per_split = static_cast<int>(cdiv(g.args.k_stages, g.splits));
   g.splits = static_cast<int>(cdiv(g.args.k_stages, g.args.stages_per_split));  // no empty splits
+  g.args.splits = g.splits;
   g.args.n_extra = g.n_extra;
   g.args.ls = ls;
   g.args.cs = cs;
@@ -464,12 +484,15 @@ ql_status qlora_linear_fwd(int64_t M, int64_t N, int64_t K, int64_t r, const uin
     if (e != cudaSuccess) return QL_ERR_CUDA;
   }
   GemmCall g;
-  g.am = A_DEQ_K;
+  g.am = A_DEQ_TMEM;
   g.b_mn = false;
   g.bn = p.bn_main;
   g.b = {x, M, K};
   if (r > 0) {
-    g.a = {B, N, r};
+    // the LoRA columns: A extra = rows of B (copied into tensor memory by the kernel), B extra = s x A^T
+    g.args.lora = B;
+    g.args.lora_ld = static_cast<int>(r);
+    g.args.lora_cols = static_cast<int>(r);
     g.bx = {su, M, r};
     g.n_extra = static_cast<int>(cdiv(r, 64));
   }

@@ -21,7 +21,7 @@ Readings: R7 -- the scaling s is lora_alpha / r ("unsloth" (pyshine.com), sectio
 Fine-Tuned Model", the ``r`` and ``lora_alpha`` arguments); the layer takes s itself.  R8 -- dY is an
 external input.  R10 -- in the gated-MLP chain the gate/up outputs and the SwiGLU output are stored as
 bf16 between the layers, as a fine-tuning framework stores activations; ``mlp_chain_*`` applies those
-roundings, ``mlp_chain_*_exact`` does not.
+roundings by default and skips them with ``round_intermediates=False``.
 
 SwiGLU ("Inside Unsloth ...", section "What You'll Learn", item "Triton Kernel Internals"; "unsloth"
 (pyshine.com), the kernels-directory paragraph naming swiglu.py):

@@ -163,7 +163,7 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
   }
   if (C::kDeq) {
     const int64_t N = g.args.w_rows, K = g.args.w_cols;
-    if (AM == A_DEQ_K || AM == A_DEQ_TMEM) {
+    if (AM == A_DEQ_TMEM) {
       if (!make_map(&tmC, g.codes, N, K / 2, 1, 32, 128, false)) return cudaErrorInvalidValue;
     } else {
       if (!make_map(&tmC, g.codes, N, K / 2, 1, 64, 64, false)) return cudaErrorInvalidValue;
@@ -204,7 +204,6 @@ cudaError_t launch_bn(const GemmCall& g, cudaStream_t stream) {
 
 cudaError_t launch_gemm(const GemmCall& g, cudaStream_t stream) {
   if (g.am == A_DEQ_TMEM && !g.b_mn) return launch_bn<A_DEQ_TMEM, false>(g, stream);
-  if (g.am == A_DEQ_K && !g.b_mn) return launch_bn<A_DEQ_K, false>(g, stream);
   if (g.am == A_DEQ_MN && !g.b_mn) return launch_bn<A_DEQ_MN, false>(g, stream);
   if (g.am == A_TMA_K && !g.b_mn) return launch_bn<A_TMA_K, false>(g, stream);
   if (g.am == A_TMA_K && g.b_mn) return launch_bn<A_TMA_K, true>(g, stream);
@@ -492,7 +491,7 @@ ql_status qlora_linear_fwd(int64_t M, int64_t N, int64_t K, int64_t r, const uin
     // the LoRA columns: A extra = rows of B (copied into tensor memory by the kernel), B extra = s x A^T
     g.args.lora = B;
     g.args.lora_ld = static_cast<int>(r);
-    g.args.lora_cols = static_cast<int>(r);
+    g.args.lora_r = static_cast<int>(r);
     g.bx = {su, M, r};
     g.n_extra = static_cast<int>(cdiv(r, 64));
   }
@@ -568,7 +567,10 @@ ql_status qlora_linear_bwd(int64_t M, int64_t N, int64_t K, int64_t r, const uin
     g.bn = p.bn_main;
     g.b = {dy, M, N};
     if (r > 0) {
-      g.a = {A, r, K};
+      // the LoRA rows: A extra = A [r, K] (copied into the MN-major tiles by the kernel), B extra = v
+      g.args.lora = A;
+      g.args.lora_ld = static_cast<int>(K);
+      g.args.lora_r = static_cast<int>(r);
       g.bx = {v, M, r};
       g.n_extra = static_cast<int>(cdiv(r, 64));
     }

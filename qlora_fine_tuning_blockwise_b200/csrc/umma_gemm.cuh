@@ -4,32 +4,44 @@
 // one split of the contraction (64-element stages), optionally preceded by "extra" stages that append the
 // rank-r LoRA columns to the contraction ([x | s u] . [deq(W) | B]^T in the forward, [dY | v] . [deq(W); A]
 // in the backward), so base and LoRA products land in one accumulator.  Each CTA walks units
-// blockIdx.x, blockIdx.x + gridDim.x, ...; its shared-memory stage ring runs on across units, and the two
-// TMEM accumulators alternate between units so the epilogue of one overlaps the mainloop of the next.
+// blockIdx.x, blockIdx.x + gridDim.x, ...; its rings run on across units, and where tensor memory allows
+// two accumulators alternate between units so the epilogue of one overlaps the mainloop of the next.
 //
 // The weight is always the 128-row (M-side) operand: the kernel computes the transposed product
 // (y^T = deq(W) x^T, dX^T = deq(W)^T dY^T), so one dequantized weight element feeds BN tokens.
 //
-// Operand A, per stage (128 rows x 64 contraction elements, bf16, 128-byte swizzled canonical layout):
-//   A_TMA_K / A_TMA_MN   loaded by TMA from a bf16 matrix (K-major or MN-major),
-//   A_DEQ_K              dequantized from NF4 codes by the dequantizer warps (forward: rows = W rows n),
-//   A_DEQ_MN             dequantized the same way into the MN-major layout (backward: rows = W columns k,
-//                        contraction over W rows n) -- the transpose of deq(W) costs nothing extra.
+// Operand A, per stage (128 rows x 64 contraction elements, bf16):
+//   A_TMA_K / A_TMA_MN   loaded by TMA from a bf16 matrix (K-major or MN-major) together with B,
+//   A_DEQ_MN             backward: dequantized from NF4 codes into the MN-major 128B-swizzled shared-memory
+//                        layout (rows = W columns k, contraction over W rows n) -- the transpose of deq(W)
+//                        costs nothing extra; the LoRA stages copy rows of A the same way,
 //   A_DEQ_TMEM           forward: dequantized rows go from registers straight into tensor memory
 //                        (tcgen05.st) and the MMA reads A there, so A never touches shared memory; the
-//                        LoRA rows of B for the extra stages are copied the same way from global memory.
-//                        Codes are expanded through a lane-replicated table of bf16 level pairs and one
-//                        bf16x2 multiply by the block scale (about two instructions per element).
-//   The codes arrive by TMA and the stage's absmax values by cp.async, both on the stage's codes barrier.
-// Operand B (BN x 64): always by TMA (K-major or MN-major).
+//                        LoRA stages copy rows of B the same way.
+// Operand B (BN x 64): always by TMA.
 //
-// Warp roles: warp 0 = producer (lane 0 issues TMA; all lanes copy absmax), warp 1 = TMEM allocator + MMA
-// issuer (one thread), warps 2..5 = epilogue (TMEM -> registers -> global), warps 6..13 = dequantizers
-// (A_DEQ_* only; two groups of 4 warps, group g takes the stages of even/odd global index).
+// Three rings decouple the latencies of the dequantizing kernels:
+//   Q ring (deep):  packed codes (TMA) + the stage's 128 absmax values (cp.async), filled by the Q producer
+//                   as far ahead as its depth allows, emptied as soon as a dequantizer has the stage in
+//                   registers -- so HBM latency overlaps many stages of work;
+//   A ring:         dequantized A tiles (TMEM columns or shared memory), filled by the dequantizers,
+//                   emptied by the MMAs (tcgen05.commit);
+//   B ring:         B tiles (and A tiles in the TMA modes), filled by the B producer, emptied by the MMAs.
+// In the dequantizing modes the MMA waits on the A ring only: a dequantizer warp arrives there after it has
+// also seen the stage's B tile land.
+//
+// Warp roles: warp 0 = B producer (lane 0 issues TMA), warp 1 = TMEM allocator + MMA issuer, warps 2..5 =
+// epilogue (TMEM -> registers -> global), warps 6 .. 6 + 4G - 1 = dequantizers (G groups of 4 warps; group
+// g % G takes stage g), warp 6 + 4G = Q producer (lane 0 issues the codes TMA, all lanes copy absmax).  The
+// dequantizer and Q-producer warps exist in the dequantizing modes only.
 //
 // Shared-memory tiles: for the 128B swizzle every tile starts on a 1024-byte boundary; row r of a tile is
 // 128 bytes at r*128 and its 16-byte chunk c sits at chunk position c ^ (r & 7).  TMA writes that layout;
 // the dequantizers write it with plain 16-byte stores followed by fence.proxy.async.
+//
+// Every wait is bounded; on expiry the waiting thread raises the CTA's abort flag and the device error word,
+// every role leaves its loop, and the producers wait (bounded) for their copies in flight before the CTA
+// releases its shared and tensor memory.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -39,7 +51,7 @@
 
 namespace qlora {
 
-enum AMode : int { A_TMA_K = 0, A_TMA_MN = 1, A_DEQ_K = 2, A_DEQ_MN = 3, A_DEQ_TMEM = 4 };
+enum AMode : int { A_TMA_K = 0, A_TMA_MN = 1, A_DEQ_MN = 3, A_DEQ_TMEM = 4 };
 
 struct UmmaArgs {
   int rows, cols;         // D extent: i in [0, rows), j in [0, cols)
@@ -51,9 +63,11 @@ struct UmmaArgs {
   // dequantization (A_DEQ_*): W is [w_rows, w_cols] with absmax [w_rows, w_cols / 64]
   const float* absmax;
   int w_rows, w_cols, w_kb;
-  // A_DEQ_TMEM extra stages: rows of the LoRA matrix appended to A ([w_rows, lora_cols], row stride lora_ld)
+  // LoRA matrix copied into the extra stages of A, row stride lora_ld, lora_r valid contraction entries:
+  //   A_DEQ_TMEM: B [w_rows, lora_r] (tile row i = W row i0 + i, contraction along the row),
+  //   A_DEQ_MN  : A [lora_r, w_cols] (contraction index = row of A, tile row i = column i0 + i).
   const uint16_t* lora;
-  int lora_ld, lora_cols;
+  int lora_ld, lora_r;
   // epilogue: out[z * split_stride + i * ls + j * cs] = alpha * D[i, j] for i < rows_lim, j < cols_lim
   void* out;
   int out_bf16;
@@ -62,7 +76,6 @@ struct UmmaArgs {
   int rows_lim, cols_lim;
   unsigned int* err;
 };
-
 
 struct Unit {
   int i0, j0, z;
@@ -90,35 +103,62 @@ __device__ __forceinline__ Unit unit_of(const UmmaArgs& a, int u, int BN) {
 template <int BN, int AM, bool B_MN>
 struct UmmaCfg {
   static constexpr bool kATmem = (AM == A_DEQ_TMEM);
-  static constexpr bool kDeq = (AM == A_DEQ_K || AM == A_DEQ_MN || kATmem);
+  static constexpr bool kDeq = (AM == A_DEQ_MN || kATmem);
   static constexpr bool kAMN = (AM == A_TMA_MN || AM == A_DEQ_MN);
-  static constexpr int kABytes = kATmem ? 0 : 128 * 64 * 2;
+  static constexpr int kTileA = 128 * 64 * 2;  // one bf16 A stage in shared memory
   static constexpr int kBBytes = BN * 64 * 2;
-  static constexpr int kCBytes = kDeq ? 4096 : 0;
-  static constexpr int kSBytes = kDeq ? 512 : 0;  // 128 absmax values per stage
-  static constexpr int kStageBytes = kABytes + kBBytes + kCBytes + kSBytes;
+  static constexpr int kBSlot = kBBytes + (kDeq ? 0 : kTileA);  // the TMA modes load A beside B
+  static constexpr int kASlot = (AM == A_DEQ_MN) ? kTileA : 0;   // A ring in shared memory
+  static constexpr int kCBytes = 4096;                            // 128 rows x 64 codes
+  static constexpr int kQSlot = kDeq ? kCBytes + 512 : 0;         // codes + 128 absmax values
   // A_DEQ_TMEM looks codes up in a shared-memory table of bf16 level pairs, one copy per lane (32 KB)
   static constexpr int kLutBytes = kATmem ? 256 * 32 * 4 : 0;
-  static constexpr int kStagesRaw = ((kATmem ? 222 : 212) * 1024 - kLutBytes) / kStageBytes;
-  static constexpr int kStagesCap = kStagesRaw > 8 ? 8 : kStagesRaw;
-  // the two dequantizer groups split the stages by index parity; with an even ring every slot keeps one group
-  static constexpr int kStages = kDeq ? (kStagesCap & ~1) : kStagesCap;
-  static constexpr int kDeqWarpsPerGroup = 4;
-  static constexpr int kThreads = 64 + 128 + (kDeq ? 256 : 0);
-  static constexpr int kAccCols = BN;  // fp32 accumulator columns per buffer
-  static constexpr int kACols = kATmem ? kStages * 32 : 0;  // A stages in TMEM: 64 bf16 = 32 columns each
-  static constexpr int kAccBufs = (2 * BN + kACols <= 512) ? 2 : 1;
+  static constexpr int kBarBytes = 1024;
+  static constexpr int kBudget = 226 * 1024 - 1024 - kLutBytes - kBarBytes;
+
+  // tensor memory: accumulators (BN fp32 columns each), then the A ring of the TMEM mode (32 columns a stage)
+  static constexpr int kAccBufs = (!kATmem || 2 * BN + 4 * 32 <= 512) ? 2 : 1;
+  static constexpr int kAccCols = BN;
   static constexpr int kAColBase = kAccBufs * BN;
-  static constexpr int kTmemNeed = kAccBufs * BN + kACols;
+  static constexpr int kAStagesTmem = (512 - kAColBase) / 32 > 8 ? 8 : (512 - kAColBase) / 32;
+
+  // ring depths.  A dequantizer's arrival waits for the stage's B tile, so the B ring bounds how far ahead the
+  // A ring may run: the A ring is never deeper than the B ring (then the B phase a dequantizer waits for is
+  // always the next one of its slot -- see the parity note in the kernel).  Deep rings when B tiles are
+  // small (token-light layers), 4 stages of 16-32 KB otherwise.
+  static constexpr int kBStagesWant = kDeq ? (BN <= 64 ? 8 : 4) : 8;
+  static constexpr int kAStagesWant = kATmem ? kAStagesTmem : (AM == A_DEQ_MN ? (BN >= 256 ? 3 : 4) : 0);
+  static constexpr int kAStages = kAStagesWant > kBStagesWant ? kBStagesWant : kAStagesWant;
+  static constexpr int kQWant = BN >= 128 ? 10 : 16;
+  static constexpr int kBFit = (kBudget - kAStages * kASlot - (kDeq ? kQWant * kQSlot : 0)) / kBSlot;
+  static constexpr int kBStages = kBFit < kBStagesWant ? (kBFit < 2 ? 2 : kBFit) : kBStagesWant;
+  static constexpr int kQFit = kDeq ? (kBudget - kAStages * kASlot - kBStages * kBSlot) / kQSlot : 0;
+  static constexpr int kQStages = kQFit > 16 ? 16 : kQFit;
+
+  // Dequantizer groups of 4 warps (one per TMEM lane quarter); group g % kDeqGroups takes stage g.  A warp
+  // spends most of a stage waiting on its own instruction latencies, so stage throughput grows with the
+  // number of groups in flight; the TMEM kernel is light on registers and runs 4, the MN-major one 2.
+  static constexpr int kDeqWarpsPerGroup = 4;
+  static constexpr int kDeqGroups = kATmem ? 4 : (kDeq ? 2 : 0);
+  static constexpr int kQWarp = 6 + 4 * kDeqGroups;
+  static constexpr int kThreads = kDeq ? 32 * (kQWarp + 1) : 64 + 128;
+  static constexpr int kTmemNeed = kAColBase + (kATmem ? kAStages * 32 : 0);
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
-  static_assert(kTmemNeed <= 512, "tensor memory");
-  static constexpr int kBarBytes = 512;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kLutBytes + kBarBytes;
+  static constexpr int kSmemBytes =
+      1024 + kBStages * kBSlot + kAStages * kASlot + kQStages * kQSlot + kLutBytes + kBarBytes;
+
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is a multiple of 16 in [16, 256]");
   static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-element swizzle atoms");
-  static_assert(kStages >= 2, "pipeline needs two stages");
+  static_assert(!(kDeq && B_MN), "the dequantizing modes take B K-major");
+  static_assert(kTmemNeed <= 512, "tensor memory");
+  static_assert(kBStages >= 2 && (!kDeq || (kAStages >= 2 && kQStages >= 4)), "ring depths");
+  // parity safety (see the kernel): A ring no deeper than the B ring, Q ring deeper than the A ring by at
+  // least the number of dequantizer groups, and no more groups than A slots
+  static_assert(!kDeq || (kAStages <= kBStages && kQStages >= kAStages + kDeqGroups && kDeqGroups <= kAStages),
+                "ring depth relations");
+  static_assert(kBStages <= 32 && kAStages <= 32 && kQStages <= 32, "armed-slot bit masks");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-  static_assert((4 * kStages + 4) * 8 + 8 <= kBarBytes, "barrier area");
+  static_assert((2 * (kBStages + kAStages + kQStages) + 4) * 8 + 8 <= kBarBytes, "barrier area");
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -183,31 +223,56 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   return true;
 }
 
+// Slot bookkeeping of a producer: which slots hold an armed phase whose copies may still be in flight, and
+// that phase's parity -- on abort the producer waits for exactly those before the CTA exits.
+struct Armed {
+  uint32_t mask = 0, par = 0;
+  __device__ __forceinline__ void set(int s, uint32_t p) {
+    mask |= 1u << s;
+    par = (par & ~(1u << s)) | (p << s);
+  }
+  __device__ __forceinline__ void drain(uint64_t* full, int n, unsigned int* err) const {
+    for (int s = 0; s < n; ++s)
+      if ((mask >> s) & 1u) mbar_wait_drain(&full[s], (par >> s) & 1u, err);
+  }
+};
+
 template <int BN, int AM, bool B_MN>
 __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC,
                      const UmmaArgs args) {
   using C = UmmaCfg<BN, AM, B_MN>;
-  constexpr int ST = C::kStages;
+  constexpr int BS = C::kBStages;
+  constexpr int AS = C::kAStages;
+  constexpr int QS = C::kQStages;
   constexpr uint32_t kFull = 0xffffffffu;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + ST * C::kABytes;
-  uint8_t* sC = sB + ST * C::kBBytes;
-  float* sS = reinterpret_cast<float*>(sC + ST * C::kCBytes);
-  uint32_t* sLut = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(sS) + ST * C::kSBytes);
-  // Barrier phases: full_tma[s] and empty[s] advance once per use of slot s (every stage); full_codes[s]
-  // and full_deq[s] once per MAIN-stage use of slot s (the LoRA stages carry no codes); tmem_full[b] and
-  // tmem_empty[b] once per unit accumulated in buffer b.  Every waiter visits every phase of the barriers
-  // it waits on, so a parity wait never aliases an older phase.
-  uint64_t* full_tma = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sLut) + C::kLutBytes);
-  uint64_t* full_codes = full_tma + ST;
-  uint64_t* full_deq = full_codes + ST;
-  uint64_t* empty = full_deq + ST;
-  uint64_t* tmem_full = empty + ST;
+  // align by pointer arithmetic on the shared array itself (not through an integer), so every pointer derived
+  // from it stays a known shared-memory pointer and compiles to shared loads and stores
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sB = smem;                          // B ring (B, then A in the TMA modes), 1024-aligned slots
+  uint8_t* sA = sB + BS * C::kBSlot;           // A ring of A_DEQ_MN, 1024-aligned slots
+  uint8_t* sQ = sA + AS * C::kASlot;           // Q ring: codes, then absmax
+  uint32_t* sLut = reinterpret_cast<uint32_t*>(sQ + QS * C::kQSlot);
+  // Phases: b_* advance once per stage (every stage uses the B ring), a_* once per stage in the dequantizing
+  // modes, q_* once per MAIN stage, tmem_* once per unit accumulated in that buffer.  Each waiter derives
+  // the parity from its running count of the ring's uses, which is sound only while the barrier's previous
+  // phase has completed when the wait starts and its next one cannot complete before the waiter releases:
+  //   - a barrier cannot run ahead: each refill needs the consumer's release of the slot first;
+  //   - a dequantizer at stage g has seen the MMAs of stage g - G - AS complete (its own previous stage's
+  //     a_empty wait, G = dequantizer groups), so with G <= AS its a_empty wait for stage g - AS cannot see
+  //     an older phase, with QS >= AS + G the Q stage QS before its own has been consumed, and (after the
+  //     a_empty wait) with AS <= BS the B stage BS before its own has landed.
+  uint64_t* b_full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sLut) + C::kLutBytes);
+  uint64_t* b_empty = b_full + BS;
+  uint64_t* a_full = b_empty + BS;
+  uint64_t* a_empty = a_full + AS;
+  uint64_t* q_full = a_empty + AS;
+  uint64_t* q_empty = q_full + QS;
+  uint64_t* tmem_full = q_empty + QS;
   uint64_t* tmem_empty = tmem_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -217,11 +282,17 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
   const int num_units = args.splits * args.tiles_i * args.tiles_j;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(&full_tma[s], 1);
-      mbar_init(&full_codes[s], 1 + 32);  // the TMA arrive + one cp.async arrive per producer lane
-      mbar_init(&full_deq[s], C::kDeqWarpsPerGroup);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < BS; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int s = 0; s < AS; ++s) {
+      mbar_init(&a_full[s], C::kDeqWarpsPerGroup);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < QS; ++s) {
+      mbar_init(&q_full[s], 1 + 32);  // the TMA arrive + one cp.async arrive per Q-producer lane
+      mbar_init(&q_empty[s], C::kDeqWarpsPerGroup);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
@@ -241,10 +312,10 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmB);
-    if (C::kDeq) tma_prefetch_desc(&tmC);
-    if (!C::kDeq || (args.n_extra > 0 && !C::kATmem)) tma_prefetch_desc(&tmA);
+    if (!C::kDeq) tma_prefetch_desc(&tmA);
     if (args.n_extra > 0) tma_prefetch_desc(&tmBx);
   }
+  if (C::kDeq && warp == C::kQWarp && lane == 0) tma_prefetch_desc(&tmC);
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -255,160 +326,104 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    uint32_t armed_tma = 0, armed_codes = 0;  // bit s: slot s has an armed phase whose copies may be in flight
-    uint32_t tma_par = 0, codes_par = 0;      // bit s: parity of that armed phase
+    // ------------------------------------------------------------------ B producer
+    Armed armed;
     int g = 0;
     bool stop = false;
     for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
       const Unit U = unit_of(args, u, BN);
       for (int it = 0; it < U.n_total; ++it, ++g) {
-        const int s = g % ST;
-        const uint32_t round = static_cast<uint32_t>(g / ST);
-        const bool ok = mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, args.err);
+        const int s = g % BS;
+        const uint32_t ph = static_cast<uint32_t>(g / BS) & 1u;
+        const bool ok = mbar_wait_idle(&b_empty[s], ph ^ 1u, abort_flag, args.err);
         if (!__all_sync(kFull, ok)) {
           stop = true;
           break;
         }
-        uint8_t* a_dst = sA + s * C::kABytes;
-        uint8_t* b_dst = sB + s * C::kBBytes;
         if (lane == 0) {
-          armed_tma |= 1u << s;
-          tma_par = (tma_par & ~(1u << s)) | ((round & 1u) << s);
-        }
-        if (it < U.n_extra && C::kATmem) {
-          // LoRA stage of the TMEM forward: B extra by TMA; the dequantizers copy A's LoRA rows themselves,
-          // so the codes barrier only counts its 33 arrivals (no bytes)
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full_tma[s], C::kBBytes);
-            tma_load_2d(b_dst, &tmBx, 64 * it, U.j0, &full_tma[s]);
-            const uint32_t cpar = ((codes_par >> s) & 1u) ^ ((armed_codes >> s) & 1u);
-            armed_codes |= 1u << s;
-            codes_par = (codes_par & ~(1u << s)) | (cpar << s);
-            mbar_arrive(&full_codes[s]);
-          }
-          mbar_arrive(&full_codes[s]);
-        } else if (it < U.n_extra) {
-          if (lane == 0) {
-            const int e = it;
-            mbar_arrive_expect_tx(&full_tma[s], C::kABytes + C::kBBytes);
-            if (C::kAMN) {
-              tma_load_2d(a_dst, &tmA, U.i0, 64 * e, &full_tma[s]);
-              tma_load_2d(a_dst + 8192, &tmA, U.i0 + 64, 64 * e, &full_tma[s]);
-            } else {
-              tma_load_2d(a_dst, &tmA, 64 * e, U.i0, &full_tma[s]);
-            }
-            tma_load_2d(b_dst, &tmBx, 64 * e, U.j0, &full_tma[s]);
-          }
-        } else {
-          const int kk0 = (U.main_begin + it - U.n_extra) * 64;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full_tma[s], C::kBBytes + (C::kDeq ? 0 : C::kABytes));
-            if (B_MN) {
-#pragma unroll
-              for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * 8192, &tmB, U.j0 + 64 * c, kk0, &full_tma[s]);
-            } else {
-              tma_load_2d(b_dst, &tmB, kk0, U.j0, &full_tma[s]);
-            }
-          }
+          armed.set(s, ph);
+          uint8_t* b_dst = sB + s * C::kBSlot;
           if constexpr (C::kDeq) {
-            // codes by TMA and the stage's 128 absmax values by cp.async, all on full_codes[s]; waiting on
-            // empty[s] above made this slot's A tile, codes and scales free to overwrite
-            if (lane == 0) {
-              const uint32_t cpar = ((codes_par >> s) & 1u) ^ ((armed_codes >> s) & 1u);
-              armed_codes |= 1u << s;
-              codes_par = (codes_par & ~(1u << s)) | (cpar << s);
-              mbar_arrive_expect_tx(&full_codes[s], C::kCBytes);
-              if constexpr (AM == A_DEQ_K || AM == A_DEQ_TMEM)
-                tma_load_2d(sC + s * C::kCBytes, &tmC, kk0 / 2, U.i0, &full_codes[s]);
-              else
-                tma_load_2d(sC + s * C::kCBytes, &tmC, U.i0 / 2, kk0, &full_codes[s]);
-            }
-            float* sdst = sS + s * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int idx = lane + 32 * q;
-              int n, k;
-              if (AM != A_DEQ_MN) {  // value for tile row idx (W row i0 + idx) in k-block kk0 / 64
-                n = U.i0 + idx;
-                k = kk0;
-              } else {              // value for W row kk0 + idx / 2 in k-block (i0 + 64 (idx & 1)) / 64
-                n = kk0 + (idx >> 1);
-                k = U.i0 + 64 * (idx & 1);
-              }
-              const bool valid = n < args.w_rows && k < args.w_cols;
-              const float* src = valid ? args.absmax + static_cast<long long>(n) * args.w_kb + (k >> 6) : args.absmax;
-              cp_async_4_zfill(sdst + idx, src, valid);
-            }
-            cp_async_mbar_arrive_noinc(&full_codes[s]);
+            mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
+            if (it < U.n_extra)
+              tma_load_2d(b_dst, &tmBx, 64 * it, U.j0, &b_full[s]);
+            else
+              tma_load_2d(b_dst, &tmB, (U.main_begin + it - U.n_extra) * 64, U.j0, &b_full[s]);
           } else {
-            if (lane == 0) {
-              if constexpr (AM == A_TMA_MN) {
-                tma_load_2d(a_dst, &tmA, U.i0, kk0, &full_tma[s]);
-                tma_load_2d(a_dst + 8192, &tmA, U.i0 + 64, kk0, &full_tma[s]);
-              } else {
-                tma_load_2d(a_dst, &tmA, kk0, U.i0, &full_tma[s]);
-              }
+            // the TMA modes have no extra stages
+            const int kk0 = (U.main_begin + it) * 64;
+            uint8_t* a_dst = b_dst + C::kBBytes;
+            mbar_arrive_expect_tx(&b_full[s], C::kBBytes + C::kTileA);
+            if constexpr (B_MN) {
+#pragma unroll
+              for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * 8192, &tmB, U.j0 + 64 * c, kk0, &b_full[s]);
+            } else {
+              tma_load_2d(b_dst, &tmB, kk0, U.j0, &b_full[s]);
+            }
+            if constexpr (AM == A_TMA_MN) {
+              tma_load_2d(a_dst, &tmA, U.i0, kk0, &b_full[s]);
+              tma_load_2d(a_dst + 8192, &tmA, U.i0 + 64, kk0, &b_full[s]);
+            } else {
+              tma_load_2d(a_dst, &tmA, kk0, U.i0, &b_full[s]);
             }
           }
         }
       }
     }
-    if (lane == 0 && *abort_flag) {
-      // copies still in flight must land before the CTA's shared memory is released: wait for the last
-      // armed phase of every slot (already complete ones return at once)
-      for (int s = 0; s < ST; ++s) {
-        if ((armed_tma >> s) & 1u) mbar_wait_drain(&full_tma[s], (tma_par >> s) & 1u, args.err);
-        if ((armed_codes >> s) & 1u) mbar_wait_drain(&full_codes[s], (codes_par >> s) & 1u, args.err);
-      }
-    }
+    // copies still in flight must land before the CTA's shared memory is released
+    if (lane == 0 && *abort_flag) armed.drain(b_full, BS, args.err);
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, C::kAMN, B_MN);
-      // full_deq[s] phases count the main-stage uses of slot s: bit s = parity of the next one
-      uint32_t deq_phase = 0;
-      int g = 0, lu = 0;
-      bool stop = false;
-      for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x, ++lu) {
-        const Unit U = unit_of(args, u, BN);
-        const int acc = lu % C::kAccBufs;
-        if (!mbar_wait(&tmem_empty[acc], (static_cast<uint32_t>(lu / C::kAccBufs) & 1u) ^ 1u, abort_flag, args.err)) break;
+    // ------------------------------------------------------------------ MMA issuer (whole warp waits,
+    // one elected lane issues)
+    constexpr uint32_t idesc = idesc_bf16_f32(128, BN, C::kAMN, B_MN);
+    int g = 0, lu = 0;
+    bool stop = false;
+    for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x, ++lu) {
+      const Unit U = unit_of(args, u, BN);
+      const int acc = lu % C::kAccBufs;
+      const uint32_t eph = (static_cast<uint32_t>(lu / C::kAccBufs) & 1u) ^ 1u;
+      if (!__all_sync(kFull, mbar_wait(&tmem_empty[acc], eph, abort_flag, args.err))) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccCols);
+      for (int it = 0; it < U.n_total; ++it, ++g) {
+        const int bs = g % BS;
+        int as = 0;
+        bool ok;
+        if constexpr (C::kDeq) {
+          // a dequantizer arrives on a_full only after the stage's B tile has landed as well
+          as = g % AS;
+          ok = mbar_wait(&a_full[as], static_cast<uint32_t>(g / AS) & 1u, abort_flag, args.err);
+        } else {
+          ok = mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err);
+        }
+        if (!__all_sync(kFull, ok)) {
+          stop = true;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccCols);
-        for (int it = 0; it < U.n_total; ++it, ++g) {
-          const int s = g % ST;
-          const uint32_t par = static_cast<uint32_t>(g / ST) & 1u;
-          if (!mbar_wait(&full_tma[s], par, abort_flag, args.err)) {
-            stop = true;
-            break;
-          }
-          if (C::kDeq && (C::kATmem || it >= U.n_extra)) {
-            if (!mbar_wait(&full_deq[s], (deq_phase >> s) & 1u, abort_flag, args.err)) {
-              stop = true;
-              break;
-            }
-            deq_phase ^= 1u << s;
-          }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + s * C::kABytes);
-          const uint32_t b0 = smem_u32(sB + s * C::kBBytes);
+        if (elect_one()) {
+          const uint32_t b0 = smem_u32(sB + bs * C::kBSlot);
+          const uint32_t a0 = C::kDeq ? smem_u32(sA + as * C::kASlot) : b0 + C::kBBytes;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint64_t bdesc = B_MN ? sdesc_sw128(b0 + k * 2048, 8192, 1024) : sdesc_sw128(b0 + k * 32, 16, 1024);
+            const uint32_t accum = (it > 0 || k > 0) ? 1u : 0u;
             if constexpr (C::kATmem) {
-              const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::kAColBase + s * 32 + k * 8);
-              umma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
+              const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::kAColBase + as * 32 + k * 8);
+              umma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, accum);
             } else {
               const uint64_t adesc =
                   C::kAMN ? sdesc_sw128(a0 + k * 2048, 8192, 1024) : sdesc_sw128(a0 + k * 32, 16, 1024);
-              umma_bf16_ss(d_tmem, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
+              umma_bf16_ss(d_tmem, adesc, bdesc, idesc, accum);
             }
           }
-          umma_commit(&empty[s]);
+          umma_commit(&b_empty[bs]);
+          if constexpr (C::kDeq) umma_commit(&a_empty[as]);
         }
-        umma_commit(&tmem_full[acc]);  // also on abort, so the MMAs already issued can be waited for
+        __syncwarp();
       }
+      if (elect_one()) umma_commit(&tmem_full[acc]);  // also on abort, so the MMAs issued can be waited for
+      __syncwarp();
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
@@ -417,7 +432,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
     for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++lu) {
       const Unit U = unit_of(args, u, BN);
       const int acc = lu % C::kAccBufs;
-      int ok = mbar_wait(&tmem_full[acc], static_cast<uint32_t>(lu / C::kAccBufs) & 1u, abort_flag, args.err) ? 1 : 0;
+      int ok = mbar_wait_idle(&tmem_full[acc], static_cast<uint32_t>(lu / C::kAccBufs) & 1u, abort_flag, args.err) ? 1 : 0;
       tc_fence_after();
       ok = __shfl_sync(kFull, ok && !*abort_flag, 0);
       if (!ok) break;
@@ -427,6 +442,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
         uint32_t r[16];
+        __syncwarp();  // tcgen05.ld is warp-aligned: reconverge after the guarded stores
         tmem_ld_32x32b_x16(t_acc + static_cast<uint32_t>(c0), r);
         tmem_ld_wait();
         if (i < args.rows_lim) {
@@ -448,108 +464,173 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tmem_empty[acc]);
     }
+  } else if (warp == C::kQWarp) {
+    // ------------------------------------------------------------------ Q producer (dequantizing modes)
+    if constexpr (C::kDeq) {
+      Armed armed;
+      int q = 0;
+      bool stop = false;
+      for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
+        const Unit U = unit_of(args, u, BN);
+        for (int it = U.n_extra; it < U.n_total; ++it, ++q) {
+          const int s = q % QS;
+          const uint32_t ph = static_cast<uint32_t>(q / QS) & 1u;
+          const bool ok = mbar_wait_idle(&q_empty[s], ph ^ 1u, abort_flag, args.err);
+          if (!__all_sync(kFull, ok)) {
+            stop = true;
+            break;
+          }
+          const int kk0 = (U.main_begin + it - U.n_extra) * 64;
+          uint8_t* q_dst = sQ + s * C::kQSlot;
+          if (lane == 0) {
+            armed.set(s, ph);
+            mbar_arrive_expect_tx(&q_full[s], C::kCBytes);
+            if constexpr (AM == A_DEQ_TMEM)
+              tma_load_2d(q_dst, &tmC, kk0 / 2, U.i0, &q_full[s]);  // 128 W rows x 32 bytes
+            else
+              tma_load_2d(q_dst, &tmC, U.i0 / 2, kk0, &q_full[s]);  // 64 W rows x 64 bytes
+          }
+          float* sdst = reinterpret_cast<float*>(q_dst + C::kCBytes);
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int idx = lane + 32 * qq;
+            int n, k;
+            if constexpr (AM == A_DEQ_TMEM) {  // value for tile row idx (W row i0 + idx) in k-block kk0 / 64
+              n = U.i0 + idx;
+              k = kk0;
+            } else {                           // value for W row kk0 + idx / 2 in k-block (i0 + 64 (idx & 1)) / 64
+              n = kk0 + (idx >> 1);
+              k = U.i0 + 64 * (idx & 1);
+            }
+            const bool valid = n < args.w_rows && k < args.w_cols;
+            const float* src = valid ? args.absmax + static_cast<long long>(n) * args.w_kb + (k >> 6) : args.absmax;
+            cp_async_4_zfill(sdst + idx, src, valid);
+          }
+          cp_async_mbar_arrive_noinc(&q_full[s]);
+        }
+      }
+      if (lane == 0 && *abort_flag) armed.drain(q_full, QS, args.err);
+    }
   } else {
-    // ------------------------------------------------------------------ dequantizers (warps 6..13)
-    if constexpr (C::kATmem) {
-      // A thread owns TMEM lane 32 * (warp % 4) + lane = tile row i (W row i0 + i) and, per stage of its
-      // group, writes that row's 64 bf16 (32 columns) into the stage's A columns of tensor memory.
-      const int grp = (warp - 6) >> 2;
-      const int row = 32 * (warp & 3) + lane;
+    // ------------------------------------------------------------------ dequantizers (warps 6 .. 6 + 4G - 1)
+    if constexpr (C::kDeq) {
+      const int t = threadIdx.x - 192;  // 0 .. 128 kDeqGroups - 1
+      const int grp = t >> 7;
+      const int tg = t & 127;
+      // A_DEQ_TMEM: thread = TMEM lane 32 (warp % 4) + lane = tile row (W row i0 + row), 64 elements a stage.
+      // A_DEQ_MN  : thread = (contraction row `row` = W row kk0 + row, half h of the 128-wide k range); rows
+      //             map so that the 8 lanes of a store phase hit 8 distinct 16-byte bank groups.
+      const int row = C::kATmem ? 32 * (warp & 3) + lane : ((tg & 7) + 8 * (tg >> 4));
+      const int h = C::kATmem ? 0 : ((tg >> 3) & 1);
+      const int c_off = C::kATmem ? row * 32 : (row * 64 + h * 32);
+      const int s_idx = C::kATmem ? row : (row * 2 + h);
       const uint32_t t_lane = static_cast<uint32_t>(32 * (warp & 3)) << 16;
       const uint8_t* lut_lane = reinterpret_cast<const uint8_t*>(sLut) + lane * 4;
-      uint32_t codes_phase = 0;  // bit s: parity of the next full_codes[s] phase (every stage of slot s)
-      int g = 0;
+      int g = 0, q = 0;
       bool stop = false;
       for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
         const Unit U = unit_of(args, u, BN);
         for (int it = 0; it < U.n_total; ++it, ++g) {
-          if ((g & 1) != grp) continue;
-          const int s = g % ST;
-          if (!mbar_wait(&full_codes[s], (codes_phase >> s) & 1u, abort_flag, args.err)) {
-            stop = true;
-            break;
-          }
-          codes_phase ^= 1u << s;
-          tc_fence_after();  // the MMAs that read this slot's A columns have completed (empty -> producer)
+          const bool extra = it < U.n_extra;
+          const int qi = q;
+          if (!extra) ++q;
+          if (g % C::kDeqGroups != grp) continue;
           uint32_t r[32];
-          if (it < U.n_extra) {
-            const int n = U.i0 + row;
-            const int c0 = 64 * it;
+          if (extra) {
+            // LoRA rows: 64 contraction entries of this thread's tile row (TMEM) or its row/half (MN)
+            const uint16_t* src;
+            bool valid;
+            if constexpr (C::kATmem) {
+              const int n = U.i0 + row;
+              valid = n < args.w_rows;
+              src = args.lora + static_cast<long long>(n) * args.lora_ld + 64 * it;
+            } else {
+              const int jr = 64 * it + row;
+              valid = jr < args.lora_r && U.i0 + 64 * h < args.w_cols;
+              src = args.lora + static_cast<long long>(jr) * args.lora_ld + U.i0 + 64 * h;
+            }
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               uint4 v = make_uint4(0, 0, 0, 0);
-              if (n < args.w_rows && c0 + 8 * c < args.lora_cols)
-                v = __ldg(reinterpret_cast<const uint4*>(args.lora + static_cast<long long>(n) * args.lora_ld + c0 + 8 * c));
+              if (valid && (!C::kATmem || 64 * it + 8 * c < args.lora_r))
+                v = __ldg(reinterpret_cast<const uint4*>(src + 8 * c));
               r[4 * c] = v.x;
               r[4 * c + 1] = v.y;
               r[4 * c + 2] = v.z;
               r[4 * c + 3] = v.w;
             }
           } else {
-            // level pair from this lane's copy of the table, times the block scale in bf16x2
-            const __nv_bfloat162 sc2 = __float2bfloat162_rn(sS[s * 128 + row]);
-            const uint4 c01 = *reinterpret_cast<const uint4*>(sC + s * C::kCBytes + row * 32);
-            const uint4 c23 = *reinterpret_cast<const uint4*>(sC + s * C::kCBytes + row * 32 + 16);
+            const int qs = qi % QS;
+            const bool okq = mbar_wait_idle(&q_full[qs], static_cast<uint32_t>(qi / QS) & 1u, abort_flag, args.err);
+            if (!__all_sync(kFull, okq)) {
+              stop = true;
+              break;
+            }
+            const uint8_t* q_src = sQ + qs * C::kQSlot;
+            const float sc = reinterpret_cast<const float*>(q_src + C::kCBytes)[s_idx];
+            const uint4 c01 = *reinterpret_cast<const uint4*>(q_src + c_off);
+            const uint4 c23 = *reinterpret_cast<const uint4*>(q_src + c_off + 16);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_empty[qs]);  // the stage is in registers: the slot may refill
             const uint32_t words[8] = {c01.x, c01.y, c01.z, c01.w, c23.x, c23.y, c23.z, c23.w};
+            if constexpr (C::kATmem) {
+              // level pair from this lane's copy of the table, times the block scale in bf16x2
+              const __nv_bfloat162 sc2 = __float2bfloat162_rn(sc);
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {
-              const uint32_t q = words[w];
-              const uint32_t offs[4] = {(q << 7) & 0x7F80u, (q >> 1) & 0x7F80u, (q >> 9) & 0x7F80u, (q >> 17) & 0x7F80u};
+              for (int w = 0; w < 8; ++w) {
+                const uint32_t qw8 = words[w];
+                const uint32_t offs[4] = {(qw8 << 7) & 0x7F80u, (qw8 >> 1) & 0x7F80u, (qw8 >> 9) & 0x7F80u,
+                                          (qw8 >> 17) & 0x7F80u};
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                uint32_t v = *reinterpret_cast<const uint32_t*>(lut_lane + offs[j]);
-                __nv_bfloat162 p = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc2);
-                r[4 * w + j] = *reinterpret_cast<uint32_t*>(&p);
+                for (int j = 0; j < 4; ++j) {
+                  uint32_t v = *reinterpret_cast<const uint32_t*>(lut_lane + offs[j]);
+                  __nv_bfloat162 p = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc2);
+                  r[4 * w + j] = *reinterpret_cast<uint32_t*>(&p);
+                }
+              }
+            } else {
+              const Nf4RegTable tab = nf4_reg_table(sc);
+#pragma unroll
+              for (int w = 0; w < 8; ++w) {
+                uint32_t o[4];
+                nf4_lookup8(tab, words[w], o);
+                r[4 * w] = o[0];
+                r[4 * w + 1] = o[1];
+                r[4 * w + 2] = o[2];
+                r[4 * w + 3] = o[3];
               }
             }
           }
-          tmem_st_32x32b_x32(tmem_base + t_lane + static_cast<uint32_t>(C::kAColBase + s * 32), r);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full_deq[s]);
-        }
-      }
-    } else if constexpr (C::kDeq) {
-      // A thread expands one 64-element block row per stage:
-      //   A_DEQ_K : thread = W row n of the stage (128 rows x 64 k), K-major tile,
-      //   A_DEQ_MN: thread = (W row n of the stage, half h of the 128-wide k range), MN-major tile;
-      //             rows map so that the 8 lanes of a store phase hit 8 distinct 16-byte bank groups.
-      const int t = threadIdx.x - 192;  // 0..255
-      const int grp = t >> 7;
-      const int tg = t & 127;
-      const int row = (AM == A_DEQ_K) ? tg : ((tg & 7) + 8 * (tg >> 4));
-      const int h = (AM == A_DEQ_K) ? 0 : ((tg >> 3) & 1);
-      const int c_off = (AM == A_DEQ_K) ? row * 32 : (row * 64 + h * 32);
-      const int a_off = (AM == A_DEQ_K) ? row * 128 : (h * 8192 + row * 128);
-      const int s_idx = (AM == A_DEQ_K) ? row : (row * 2 + h);
-      uint32_t codes_phase = 0;  // bit s: parity of the next full_codes[s] phase (this group owns slot s)
-      int g = 0;
-      bool stop = false;
-      for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
-        const Unit U = unit_of(args, u, BN);
-        for (int it = 0; it < U.n_total; ++it, ++g) {
-          if (it < U.n_extra || (g & 1) != grp) continue;
-          const int s = g % ST;
-          if (!mbar_wait(&full_codes[s], (codes_phase >> s) & 1u, abort_flag, args.err)) {
+          // the A slot is free once the MMAs of its previous stage have completed
+          const int as = g % AS;
+          const bool oka = mbar_wait_idle(&a_empty[as], (static_cast<uint32_t>(g / AS) & 1u) ^ 1u, abort_flag, args.err);
+          if (!__all_sync(kFull, oka)) {
             stop = true;
             break;
           }
-          codes_phase ^= 1u << s;
-          const Nf4RegTable tab = nf4_reg_table(sS[s * 128 + s_idx]);
-          const uint4 c01 = *reinterpret_cast<const uint4*>(sC + s * C::kCBytes + c_off);
-          const uint4 c23 = *reinterpret_cast<const uint4*>(sC + s * C::kCBytes + c_off + 16);
-          const uint32_t words[8] = {c01.x, c01.y, c01.z, c01.w, c23.x, c23.y, c23.z, c23.w};
-          uint8_t* a_row = sA + s * C::kABytes + a_off;
+          tc_fence_after();
+          if constexpr (C::kATmem) {
+            tmem_st_32x32b_x32(tmem_base + t_lane + static_cast<uint32_t>(C::kAColBase + as * 32), r);
+            tmem_st_wait();
+            tc_fence_before();
+          } else {
+            uint8_t* a_row = sA + as * C::kASlot + h * 8192 + row * 128;
 #pragma unroll
-          for (int w = 0; w < 8; ++w) {
-            uint32_t o[4];
-            nf4_lookup8(tab, words[w], o);
-            *reinterpret_cast<uint4*>(a_row + ((w ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            for (int w = 0; w < 8; ++w)
+              *reinterpret_cast<uint4*>(a_row + ((w ^ (row & 7)) << 4)) =
+                  make_uint4(r[4 * w], r[4 * w + 1], r[4 * w + 2], r[4 * w + 3]);
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&full_deq[s]);
+          if (lane == 0) {
+            // the MMA waits on a_full alone: arrive only once the stage's B tile has landed as well
+            const int bs = g % BS;
+            bool okb = mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err);
+            if (okb) mbar_arrive(&a_full[as]);
+            else stop = true;
+          }
+          stop = __shfl_sync(kFull, stop ? 1 : 0, 0) != 0;
+          if (stop) break;
         }
       }
     }

@@ -417,8 +417,9 @@ def oracle_step_sample(workload: str, m_sample: int):
     return dt, flops
 
 
-def cpu_baseline(workload: str, target_s: float = 12.0) -> dict:
-    """The oracle as it stands, on a sub-batch sized for about `target_s` seconds of host work."""
+def cpu_baseline(workload: str, target_s: float = 12.0, max_steps: int = 60) -> dict:
+    """The oracle as it stands, on a bounded sample of about `target_s` seconds of host work: a token sub-batch
+    when one full step would take longer, else whole steps repeated until the target (at most `max_steps`)."""
     from qlora_fine_tuning_blockwise_b200 import inputs as I
     M = I.WORKLOADS[workload].M
     dt, flops = oracle_step_sample(workload, min(256, M))
@@ -426,9 +427,15 @@ def cpu_baseline(workload: str, target_s: float = 12.0) -> dict:
     m_sample -= m_sample % 64 if m_sample > 64 else 0
     if m_sample != min(256, M):
         dt, flops = oracle_step_sample(workload, m_sample)
-    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{workload} with the first {m_sample} of its tokens: dequantize + fwd + bwd in fp64 "
-                      f"(numpy), {dt:.2f} s", "seconds": round(dt, 3)}
+    steps, tot_t, tot_f = 1, dt, flops
+    while tot_t < target_s and steps < max_steps:
+        dt, flops = oracle_step_sample(workload, m_sample)
+        tot_t += dt
+        tot_f += flops
+        steps += 1
+    return {"value": round(tot_f / tot_t / 1e12, 5), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{workload}, first {m_sample} of its {M} tokens, {steps} step(s) of dequantize + fwd + bwd "
+                      f"in fp64 (numpy), {tot_t:.1f} s timed", "seconds": round(tot_t, 3)}
 
 
 def run_reference(args):

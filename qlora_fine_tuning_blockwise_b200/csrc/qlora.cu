@@ -99,7 +99,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major matrix [rows, cols] of 1- or 2-byte elements; box = box_cols x box_rows.
+// Row-major matrix [rows, cols] of 1-, 2- or 4-byte elements; box = box_cols x box_rows.
 bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
               int box_rows, bool swizzle128) {
   EncodeTiledFn fn = encode_fn();
@@ -108,7 +108,10 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
   cuuint64_t gstride[1] = {static_cast<cuuint64_t>(cols * elem_bytes)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+  const CUtensorMapDataType dt = elem_bytes == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = fn(m, dt, 2,
                   const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -130,15 +133,16 @@ struct GemmCall {
   const uint8_t* codes = nullptr;
   int64_t rows = 0, cols = 0, k_total = 0;
   int n_extra = 0;
+  int kb = 1;             // NF4 blocks per pipeline stage (4 only for token-light A_DEQ_TMEM)
   int splits = 1;
   int prof = -1;          // profiling-event slot recorded around this launch (-1: none)
   int ctas = 148;         // persistent CTAs: at most one per SM
   UmmaArgs args{};
 };
 
-template <int BN, int AM, bool BMN>
+template <int BN, int AM, bool BMN, int KB = 1>
 cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
-  using C = UmmaCfg<BN, AM, BMN>;
+  using C = UmmaCfg<BN, AM, BMN, KB>;
   CUtensorMap tmA, tmB, tmBx, tmC;
   std::memset(&tmA, 0, sizeof(tmA));
   std::memset(&tmBx, 0, sizeof(tmBx));
@@ -161,7 +165,12 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
   if (g.bx.ptr) {
     if (!make_map(&tmBx, g.bx.ptr, g.bx.rows, g.bx.cols, 2, 64, BN, true)) return cudaErrorInvalidValue;
   }
-  if (C::kDeq) {
+  if (C::kAbsTma) {
+    // 4-block stages: codes 128 rows x 128 bytes (swizzled), absmax 128 rows x 4 values into tmA
+    const int64_t N = g.args.w_rows, K = g.args.w_cols;
+    if (!make_map(&tmC, g.codes, N, K / 2, 1, 128, 128, true)) return cudaErrorInvalidValue;
+    if (!make_map(&tmA, g.args.absmax, N, K / 64, 4, 4, 128, false)) return cudaErrorInvalidValue;
+  } else if (C::kDeq) {
     const int64_t N = g.args.w_rows, K = g.args.w_cols;
     if (AM == A_DEQ_TMEM) {
       if (!make_map(&tmC, g.codes, N, K / 2, 1, 32, 128, false)) return cudaErrorInvalidValue;
@@ -169,7 +178,7 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
       if (!make_map(&tmC, g.codes, N, K / 2, 1, 64, 64, false)) return cudaErrorInvalidValue;
     }
   }
-  auto kern = umma_gemm_kernel<BN, AM, BMN>;
+  auto kern = umma_gemm_kernel<BN, AM, BMN, KB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int64_t units = static_cast<int64_t>(g.args.splits) * g.args.tiles_i * g.args.tiles_j;
@@ -203,6 +212,15 @@ cudaError_t launch_bn(const GemmCall& g, cudaStream_t stream) {
 }
 
 cudaError_t launch_gemm(const GemmCall& g, cudaStream_t stream) {
+  if (g.am == A_DEQ_TMEM && !g.b_mn && g.kb == 4) {
+    switch (g.bn) {
+      case 16: return launch_umma<16, A_DEQ_TMEM, false, 4>(g, stream);
+      case 32: return launch_umma<32, A_DEQ_TMEM, false, 4>(g, stream);
+      case 64: return launch_umma<64, A_DEQ_TMEM, false, 4>(g, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (g.kb != 1) return cudaErrorInvalidValue;
   if (g.am == A_DEQ_TMEM && !g.b_mn) return launch_bn<A_DEQ_TMEM, false>(g, stream);
   if (g.am == A_DEQ_MN && !g.b_mn) return launch_bn<A_DEQ_MN, false>(g, stream);
   if (g.am == A_TMA_K && !g.b_mn) return launch_bn<A_TMA_K, false>(g, stream);
@@ -249,6 +267,10 @@ int plan_splits_streaming(int64_t tiles, int64_t kstages, int sms) {
   return best;
 }
 
+// NF4 blocks per stage of the fused forward: 4 for token-light layers (short MMAs, so per-stage sync costs
+// dominate) when the absmax rows are whole 16-byte TMA boxes (K a multiple of 256), else 1.
+int fwd_stage_blocks(int64_t M, int64_t K) { return (main_bn(M) <= 64 && K % 256 == 0) ? 4 : 1; }
+
 struct LinearPlan {
   int bn_main = 16, s_main = 1;      // forward y / backward dX
   int s_su = 1, s_v = 1, s_da = 1, s_db = 1;
@@ -262,7 +284,7 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass)
   const int rp = rank_pad(r);
   p.bn_main = main_bn(M);
   const int64_t main_tiles = cdiv(M, p.bn_main) * (pass == QL_PASS_FWD ? cdiv(N, 128) : cdiv(K, 128));
-  const int64_t main_kst = pass == QL_PASS_FWD ? cdiv(K, 64) : cdiv(N, 64);
+  const int64_t main_kst = pass == QL_PASS_FWD ? cdiv(K, 64 * fwd_stage_blocks(M, K)) : cdiv(N, 64);
   p.s_main = M <= 64 ? plan_splits_streaming(main_tiles, main_kst, sms) : plan_splits(main_tiles, main_kst, sms);
   size_t part = 0;
   if (p.s_main > 1) part = std::max(part, static_cast<size_t>(p.s_main) * M * (pass == QL_PASS_FWD ? N : K) * 4);
@@ -313,7 +335,7 @@ cudaError_t run_gemm(GemmCall g, void* out, bool out_bf16, float alpha, int64_t 
   g.args.cols = static_cast<int>(g.cols);
   g.args.tiles_i = static_cast<int>(cdiv(g.rows, 128));
   g.args.tiles_j = static_cast<int>(cdiv(g.cols, g.bn));
-  g.args.k_stages = static_cast<int>(cdiv(g.k_total, 64));
+  g.args.k_stages = static_cast<int>(cdiv(g.k_total, 64 * g.kb));
   g.args.stages_per_split = static_cast<int>(cdiv(g.args.k_stages, g.splits));
   g.splits = static_cast<int>(cdiv(g.args.k_stages, g.args.stages_per_split));  // no empty splits
   g.args.splits = g.splits;
@@ -493,8 +515,9 @@ ql_status qlora_linear_fwd(int64_t M, int64_t N, int64_t K, int64_t r, const uin
     g.args.lora_ld = static_cast<int>(r);
     g.args.lora_r = static_cast<int>(r);
     g.bx = {su, M, r};
-    g.n_extra = static_cast<int>(cdiv(r, 64));
   }
+  g.kb = fwd_stage_blocks(M, K);
+  if (r > 0) g.n_extra = static_cast<int>(cdiv(r, 64 * g.kb));
   g.codes = codes;
   g.args.absmax = absmax;
   g.args.w_rows = static_cast<int>(N);

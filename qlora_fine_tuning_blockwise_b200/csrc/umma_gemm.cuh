@@ -100,17 +100,23 @@ __device__ __forceinline__ Unit unit_of(const UmmaArgs& a, int u, int BN) {
   return U;
 }
 
-template <int BN, int AM, bool B_MN>
+// KB = NF4 blocks (64 contraction elements each) per pipeline stage.  Every stage costs each role a few
+// barrier round trips of fixed latency, so token-light layers -- whose MMAs are short -- run 4 blocks a stage
+// (A_DEQ_TMEM only): codes then arrive as one 128B-swizzled TMA box of 128 rows x 128 bytes and the absmax
+// values as one TMA box of 128 rows x 4 floats.
+template <int BN, int AM, bool B_MN, int KB = 1>
 struct UmmaCfg {
   static constexpr bool kATmem = (AM == A_DEQ_TMEM);
   static constexpr bool kDeq = (AM == A_DEQ_MN || kATmem);
   static constexpr bool kAMN = (AM == A_TMA_MN || AM == A_DEQ_MN);
-  static constexpr int kTileA = 128 * 64 * 2;  // one bf16 A stage in shared memory
-  static constexpr int kBBytes = BN * 64 * 2;
+  static constexpr bool kAbsTma = (KB == 4);  // absmax by TMA (else one cp.async per row)
+  static constexpr int kTileA = 128 * 64 * 2;  // one bf16 A block in shared memory
+  static constexpr int kBBytes = BN * 64 * 2 * KB;
   static constexpr int kBSlot = kBBytes + (kDeq ? 0 : kTileA);  // the TMA modes load A beside B
   static constexpr int kASlot = (AM == A_DEQ_MN) ? kTileA : 0;   // A ring in shared memory
-  static constexpr int kCBytes = 4096;                            // 128 rows x 64 codes
-  static constexpr int kQSlot = kDeq ? kCBytes + 512 : 0;         // codes + 128 absmax values
+  static constexpr int kCBytes = 4096 * KB;                       // 128 rows x 64 KB codes
+  static constexpr int kSBytes = 512 * KB;                        // 128 rows x KB absmax values
+  static constexpr int kQSlot = kDeq ? kCBytes + kSBytes : 0;
   // A_DEQ_TMEM looks codes up in a shared-memory table of bf16 level pairs, one copy per lane (32 KB)
   static constexpr int kLutBytes = kATmem ? 256 * 32 * 4 : 0;
   static constexpr int kBarBytes = 1024;
@@ -120,7 +126,8 @@ struct UmmaCfg {
   static constexpr int kAccBufs = (!kATmem || 2 * BN + 4 * 32 <= 512) ? 2 : 1;
   static constexpr int kAccCols = BN;
   static constexpr int kAColBase = kAccBufs * BN;
-  static constexpr int kAStagesTmem = (512 - kAColBase) / 32 > 8 ? 8 : (512 - kAColBase) / 32;
+  static constexpr int kAColsStage = 32 * KB;
+  static constexpr int kAStagesTmem = (512 - kAColBase) / kAColsStage > 8 ? 8 : (512 - kAColBase) / kAColsStage;
 
   // ring depths.  A dequantizer's arrival waits for the stage's B tile, so the B ring bounds how far ahead the
   // A ring may run: the A ring is never deeper than the B ring (then the B phase a dequantizer waits for is
@@ -128,10 +135,10 @@ struct UmmaCfg {
   // small (token-light layers), 4 stages of 16-32 KB otherwise.
   static constexpr int kBStagesWant = kDeq ? (BN <= 64 ? 8 : 4) : 8;
   static constexpr int kAStagesWant = kATmem ? kAStagesTmem : (AM == A_DEQ_MN ? (BN >= 256 ? 3 : 4) : 0);
-  static constexpr int kAStages = kAStagesWant > kBStagesWant ? kBStagesWant : kAStagesWant;
-  static constexpr int kQWant = BN >= 128 ? 10 : 16;
-  static constexpr int kBFit = (kBudget - kAStages * kASlot - (kDeq ? kQWant * kQSlot : 0)) / kBSlot;
+  static constexpr int kQWant = KB == 4 ? 6 : (BN >= 128 ? 10 : 16);
+  static constexpr int kBFit = (kBudget - kAStagesWant * kASlot - (kDeq ? kQWant * kQSlot : 0)) / kBSlot;
   static constexpr int kBStages = kBFit < kBStagesWant ? (kBFit < 2 ? 2 : kBFit) : kBStagesWant;
+  static constexpr int kAStages = kAStagesWant > kBStages ? kBStages : kAStagesWant;
   static constexpr int kQFit = kDeq ? (kBudget - kAStages * kASlot - kBStages * kBSlot) / kQSlot : 0;
   static constexpr int kQStages = kQFit > 16 ? 16 : kQFit;
 
@@ -139,10 +146,10 @@ struct UmmaCfg {
   // spends most of a stage waiting on its own instruction latencies, so stage throughput grows with the
   // number of groups in flight; the TMEM kernel is light on registers and runs 4, the MN-major one 2.
   static constexpr int kDeqWarpsPerGroup = 4;
-  static constexpr int kDeqGroups = kATmem ? 4 : (kDeq ? 2 : 0);
+  static constexpr int kDeqGroups = kATmem ? (kAStages < 4 ? kAStages : 4) : (kDeq ? 2 : 0);
   static constexpr int kQWarp = 6 + 4 * kDeqGroups;
   static constexpr int kThreads = kDeq ? 32 * (kQWarp + 1) : 64 + 128;
-  static constexpr int kTmemNeed = kAColBase + (kATmem ? kAStages * 32 : 0);
+  static constexpr int kTmemNeed = kAColBase + (kATmem ? kAStages * kAColsStage : 0);
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kSmemBytes =
       1024 + kBStages * kBSlot + kAStages * kASlot + kQStages * kQSlot + kLutBytes + kBarBytes;
@@ -150,6 +157,7 @@ struct UmmaCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is a multiple of 16 in [16, 256]");
   static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-element swizzle atoms");
   static_assert(!(kDeq && B_MN), "the dequantizing modes take B K-major");
+  static_assert(KB == 1 || (kATmem && KB == 4), "4-block stages exist for the TMEM forward only");
   static_assert(kTmemNeed <= 512, "tensor memory");
   static_assert(kBStages >= 2 && (!kDeq || (kAStages >= 2 && kQStages >= 4)), "ring depths");
   // parity safety (see the kernel): A ring no deeper than the B ring, Q ring deeper than the A ring by at
@@ -237,12 +245,13 @@ struct Armed {
   }
 };
 
-template <int BN, int AM, bool B_MN>
-__global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
+// tmA: A for the TMA modes; the absmax matrix [w_rows, w_cols / 64] (fp32) for 4-block TMEM stages.
+template <int BN, int AM, bool B_MN, int KB = 1>
+__global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC,
                      const UmmaArgs args) {
-  using C = UmmaCfg<BN, AM, B_MN>;
+  using C = UmmaCfg<BN, AM, B_MN, KB>;
   constexpr int BS = C::kBStages;
   constexpr int AS = C::kAStages;
   constexpr int QS = C::kQStages;
@@ -291,7 +300,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
       mbar_init(&a_empty[s], 1);
     }
     for (int s = 0; s < QS; ++s) {
-      mbar_init(&q_full[s], 1 + 32);  // the TMA arrive + one cp.async arrive per Q-producer lane
+      mbar_init(&q_full[s], C::kAbsTma ? 1 : 1 + 32);  // the TMA arrive (+ one cp.async arrive per producer lane)
       mbar_init(&q_empty[s], C::kDeqWarpsPerGroup);
     }
     for (int b = 0; b < 2; ++b) {
@@ -315,7 +324,10 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
     if (!C::kDeq) tma_prefetch_desc(&tmA);
     if (args.n_extra > 0) tma_prefetch_desc(&tmBx);
   }
-  if (C::kDeq && warp == C::kQWarp && lane == 0) tma_prefetch_desc(&tmC);
+  if (C::kDeq && warp == C::kQWarp && lane == 0) {
+    tma_prefetch_desc(&tmC);
+    if (C::kAbsTma) tma_prefetch_desc(&tmA);
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -344,11 +356,16 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
           armed.set(s, ph);
           uint8_t* b_dst = sB + s * C::kBSlot;
           if constexpr (C::kDeq) {
+            // KB blocks of BN x 64, each a 128B-swizzled K-major sub-tile
             mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
-            if (it < U.n_extra)
-              tma_load_2d(b_dst, &tmBx, 64 * it, U.j0, &b_full[s]);
-            else
-              tma_load_2d(b_dst, &tmB, (U.main_begin + it - U.n_extra) * 64, U.j0, &b_full[s]);
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+              if (it < U.n_extra)
+                tma_load_2d(b_dst + kb * BN * 128, &tmBx, 64 * (KB * it + kb), U.j0, &b_full[s]);
+              else
+                tma_load_2d(b_dst + kb * BN * 128, &tmB, ((U.main_begin + it - U.n_extra) * KB + kb) * 64, U.j0,
+                            &b_full[s]);
+            }
           } else {
             // the TMA modes have no extra stages
             const int kk0 = (U.main_begin + it) * 64;
@@ -405,11 +422,14 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
           const uint32_t b0 = smem_u32(sB + bs * C::kBSlot);
           const uint32_t a0 = C::kDeq ? smem_u32(sA + as * C::kASlot) : b0 + C::kBBytes;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t bdesc = B_MN ? sdesc_sw128(b0 + k * 2048, 8192, 1024) : sdesc_sw128(b0 + k * 32, 16, 1024);
-            const uint32_t accum = (it > 0 || k > 0) ? 1u : 0u;
+          for (int kk = 0; kk < 4 * KB; ++kk) {
+            const int kb = kk >> 2, k = kk & 3;
+            const uint32_t bk = b0 + static_cast<uint32_t>(kb * BN * 128);
+            const uint64_t bdesc = B_MN ? sdesc_sw128(bk + k * 2048, 8192, 1024) : sdesc_sw128(bk + k * 32, 16, 1024);
+            const uint32_t accum = (it > 0 || kk > 0) ? 1u : 0u;
             if constexpr (C::kATmem) {
-              const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::kAColBase + as * 32 + k * 8);
+              const uint32_t a_tmem =
+                  tmem_base + static_cast<uint32_t>(C::kAColBase + as * C::kAColsStage + kb * 32 + k * 8);
               umma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, accum);
             } else {
               const uint64_t adesc =
@@ -480,16 +500,24 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
             stop = true;
             break;
           }
-          const int kk0 = (U.main_begin + it - U.n_extra) * 64;
+          const int kk0 = (U.main_begin + it - U.n_extra) * 64 * KB;
           uint8_t* q_dst = sQ + s * C::kQSlot;
           if (lane == 0) {
             armed.set(s, ph);
-            mbar_arrive_expect_tx(&q_full[s], C::kCBytes);
-            if constexpr (AM == A_DEQ_TMEM)
-              tma_load_2d(q_dst, &tmC, kk0 / 2, U.i0, &q_full[s]);  // 128 W rows x 32 bytes
-            else
-              tma_load_2d(q_dst, &tmC, U.i0 / 2, kk0, &q_full[s]);  // 64 W rows x 64 bytes
+            if constexpr (C::kAbsTma) {
+              // 128 W rows x 128 bytes of codes (swizzled) and 128 rows x 4 absmax values
+              mbar_arrive_expect_tx(&q_full[s], C::kCBytes + C::kSBytes);
+              tma_load_2d(q_dst, &tmC, kk0 / 2, U.i0, &q_full[s]);
+              tma_load_2d(q_dst + C::kCBytes, &tmA, kk0 / 64, U.i0, &q_full[s]);
+            } else {
+              mbar_arrive_expect_tx(&q_full[s], C::kCBytes);
+              if constexpr (AM == A_DEQ_TMEM)
+                tma_load_2d(q_dst, &tmC, kk0 / 2, U.i0, &q_full[s]);  // 128 W rows x 32 bytes
+              else
+                tma_load_2d(q_dst, &tmC, U.i0 / 2, kk0, &q_full[s]);  // 64 W rows x 64 bytes
+            }
           }
+          if constexpr (C::kAbsTma) continue;
           float* sdst = reinterpret_cast<float*>(q_dst + C::kCBytes);
 #pragma unroll
           for (int qq = 0; qq < 4; ++qq) {
@@ -535,31 +563,11 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
           const int qi = q;
           if (!extra) ++q;
           if (g % C::kDeqGroups != grp) continue;
-          uint32_t r[32];
-          if (extra) {
-            // LoRA rows: 64 contraction entries of this thread's tile row (TMEM) or its row/half (MN)
-            const uint16_t* src;
-            bool valid;
-            if constexpr (C::kATmem) {
-              const int n = U.i0 + row;
-              valid = n < args.w_rows;
-              src = args.lora + static_cast<long long>(n) * args.lora_ld + 64 * it;
-            } else {
-              const int jr = 64 * it + row;
-              valid = jr < args.lora_r && U.i0 + 64 * h < args.w_cols;
-              src = args.lora + static_cast<long long>(jr) * args.lora_ld + U.i0 + 64 * h;
-            }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (valid && (!C::kATmem || 64 * it + 8 * c < args.lora_r))
-                v = __ldg(reinterpret_cast<const uint4*>(src + 8 * c));
-              r[4 * c] = v.x;
-              r[4 * c + 1] = v.y;
-              r[4 * c + 2] = v.z;
-              r[4 * c + 3] = v.w;
-            }
-          } else {
+          // The stage's codes and scales, held in registers: block p of the stage is words[8p .. 8p + 7]
+          // (64 codes) with scale sc[p].
+          uint32_t words[8 * KB];
+          float sc[KB];
+          if (!extra) {
             const int qs = qi % QS;
             const bool okq = mbar_wait_idle(&q_full[qs], static_cast<uint32_t>(qi / QS) & 1u, abort_flag, args.err);
             if (!__all_sync(kFull, okq)) {
@@ -567,40 +575,97 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
               break;
             }
             const uint8_t* q_src = sQ + qs * C::kQSlot;
-            const float sc = reinterpret_cast<const float*>(q_src + C::kCBytes)[s_idx];
-            const uint4 c01 = *reinterpret_cast<const uint4*>(q_src + c_off);
-            const uint4 c23 = *reinterpret_cast<const uint4*>(q_src + c_off + 16);
+            if constexpr (C::kAbsTma) {
+              // row `row` is 128 bytes; its 16-byte chunk c sits at chunk position c ^ (row & 7)
+              const uint8_t* q_row = q_src + row * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(q_row + ((c ^ (row & 7)) << 4));
+                words[4 * c] = v.x;
+                words[4 * c + 1] = v.y;
+                words[4 * c + 2] = v.z;
+                words[4 * c + 3] = v.w;
+              }
+              const float4 s4 = *reinterpret_cast<const float4*>(q_src + C::kCBytes + row * 16);
+              sc[0] = s4.x;
+              if constexpr (KB == 4) {
+                sc[1] = s4.y;
+                sc[2] = s4.z;
+                sc[3] = s4.w;
+              }
+            } else {
+              sc[0] = reinterpret_cast<const float*>(q_src + C::kCBytes)[s_idx];
+              const uint4 c01 = *reinterpret_cast<const uint4*>(q_src + c_off);
+              const uint4 c23 = *reinterpret_cast<const uint4*>(q_src + c_off + 16);
+              words[0] = c01.x;
+              words[1] = c01.y;
+              words[2] = c01.z;
+              words[3] = c01.w;
+              words[4] = c23.x;
+              words[5] = c23.y;
+              words[6] = c23.z;
+              words[7] = c23.w;
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&q_empty[qs]);  // the stage is in registers: the slot may refill
-            const uint32_t words[8] = {c01.x, c01.y, c01.z, c01.w, c23.x, c23.y, c23.z, c23.w};
-            if constexpr (C::kATmem) {
+          }
+          // 64 bf16 values (32 registers) of block p: dequantized codes, or the LoRA rows in the extra stages
+          auto block_values = [&](int p, uint32_t (&r)[32]) {
+            if (extra) {
+              // LoRA rows: 64 contraction entries of this thread's tile row (TMEM) or its row/half (MN)
+              const uint16_t* src;
+              bool valid;
+              int c0 = 0;
+              if constexpr (C::kATmem) {
+                const int n = U.i0 + row;
+                c0 = 64 * (KB * it + p);
+                valid = n < args.w_rows;
+                src = args.lora + static_cast<long long>(n) * args.lora_ld + c0;
+              } else {
+                const int jr = 64 * it + row;
+                valid = jr < args.lora_r && U.i0 + 64 * h < args.w_cols;
+                src = args.lora + static_cast<long long>(jr) * args.lora_ld + U.i0 + 64 * h;
+              }
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (valid && (!C::kATmem || c0 + 8 * c < args.lora_r))
+                  v = __ldg(reinterpret_cast<const uint4*>(src + 8 * c));
+                r[4 * c] = v.x;
+                r[4 * c + 1] = v.y;
+                r[4 * c + 2] = v.z;
+                r[4 * c + 3] = v.w;
+              }
+            } else if constexpr (C::kATmem) {
               // level pair from this lane's copy of the table, times the block scale in bf16x2
-              const __nv_bfloat162 sc2 = __float2bfloat162_rn(sc);
+              const __nv_bfloat162 sc2 = __float2bfloat162_rn(sc[p]);
 #pragma unroll
               for (int w = 0; w < 8; ++w) {
-                const uint32_t qw8 = words[w];
+                const uint32_t qw8 = words[8 * p + w];
                 const uint32_t offs[4] = {(qw8 << 7) & 0x7F80u, (qw8 >> 1) & 0x7F80u, (qw8 >> 9) & 0x7F80u,
                                           (qw8 >> 17) & 0x7F80u};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                   uint32_t v = *reinterpret_cast<const uint32_t*>(lut_lane + offs[j]);
-                  __nv_bfloat162 p = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc2);
-                  r[4 * w + j] = *reinterpret_cast<uint32_t*>(&p);
+                  __nv_bfloat162 pr = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc2);
+                  r[4 * w + j] = *reinterpret_cast<uint32_t*>(&pr);
                 }
               }
             } else {
-              const Nf4RegTable tab = nf4_reg_table(sc);
+              const Nf4RegTable tab = nf4_reg_table(sc[p]);
 #pragma unroll
               for (int w = 0; w < 8; ++w) {
                 uint32_t o[4];
-                nf4_lookup8(tab, words[w], o);
+                nf4_lookup8(tab, words[8 * p + w], o);
                 r[4 * w] = o[0];
                 r[4 * w + 1] = o[1];
                 r[4 * w + 2] = o[2];
                 r[4 * w + 3] = o[3];
               }
             }
-          }
+          };
+          uint32_t r[32];
+          block_values(0, r);
           // the A slot is free once the MMAs of its previous stage have completed
           const int as = g % AS;
           const bool oka = mbar_wait_idle(&a_empty[as], (static_cast<uint32_t>(g / AS) & 1u) ^ 1u, abort_flag, args.err);
@@ -610,7 +675,13 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN>::kThreads, 1)
           }
           tc_fence_after();
           if constexpr (C::kATmem) {
-            tmem_st_32x32b_x32(tmem_base + t_lane + static_cast<uint32_t>(C::kAColBase + as * 32), r);
+            const uint32_t a_col = tmem_base + t_lane + static_cast<uint32_t>(C::kAColBase + as * C::kAColsStage);
+            tmem_st_32x32b_x32(a_col, r);
+#pragma unroll
+            for (int p = 1; p < KB; ++p) {
+              block_values(p, r);
+              tmem_st_32x32b_x32(a_col + static_cast<uint32_t>(32 * p), r);
+            }
             tmem_st_wait();
             tc_fence_before();
           } else {

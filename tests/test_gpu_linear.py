@@ -67,6 +67,10 @@ SMALL = [
     (257, 512, 640, 64),
     (33, 1024, 1984, 8),    # K % 128 == 64: half-empty transposed tile in dX
     (520, 128, 128, 256),   # largest rank
+    # token-light layers with K % 256 == 0 run the forward in stages of four NF4 blocks
+    (1, 264, 512, 16),      # BN = 16, ragged N tile
+    (40, 136, 768, 72),     # BN = 64, odd number of 4-block stages, partly filled LoRA stage
+    (20, 128, 1280, 256),   # BN = 32, largest rank in one 256-wide LoRA stage
 ]
 
 
@@ -99,9 +103,11 @@ def test_tiny_workload_full(ops):
         assert_close(got[k], ref[k], k)
 
 
-def test_B_zero_equals_plain_layer_bitwise(ops):
-    """B = 0 appends products that are all zero: y must equal the r = 0 layer bit for bit."""
-    d = I.make_random_linear(200, 384, 512, 16, seed=5)
+@pytest.mark.parametrize("M", [200, 16])
+def test_B_zero_equals_plain_layer_bitwise(ops, M):
+    """B = 0 appends products that are all zero: y must equal the r = 0 layer bit for bit (M = 16 takes the
+    4-block stages of the token-light forward)."""
+    d = I.make_random_linear(M, 384, 512, 16, seed=5)
     codes, absmax = ops.nf4_quantize(dev(d["W"]))
     x = dev(d["x"])
     A = dev(d["A"])

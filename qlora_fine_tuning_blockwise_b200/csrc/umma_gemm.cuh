@@ -117,7 +117,8 @@ struct UmmaCfg {
   static constexpr int kCBytes = 4096 * KB;                       // 128 rows x 64 KB codes
   static constexpr int kSBytes = 512 * KB;                        // 128 rows x KB absmax values
   static constexpr int kQSlot = kDeq ? kCBytes + kSBytes : 0;
-  // A_DEQ_TMEM looks codes up in a shared-memory table of bf16 level pairs, one copy per lane (32 KB)
+  // the TMEM dequantizers look codes up in a shared-memory table of bf16 level pairs, one copy per lane
+  // (32 KB); the MN-major ones use a per-thread register table (exact, no shared-memory reads)
   static constexpr int kLutBytes = kATmem ? 256 * 32 * 4 : 0;
   static constexpr int kBarBytes = 1024;
   static constexpr int kBudget = 226 * 1024 - 1024 - kLutBytes - kBarBytes;
@@ -144,9 +145,9 @@ struct UmmaCfg {
 
   // Dequantizer groups of 4 warps (one per TMEM lane quarter); group g % kDeqGroups takes stage g.  A warp
   // spends most of a stage waiting on its own instruction latencies, so stage throughput grows with the
-  // number of groups in flight; the TMEM kernel is light on registers and runs 4, the MN-major one 2.
+  // number of groups in flight, up to the A ring's depth: 4 in the TMEM kernel, 2 in the MN-major one.
   static constexpr int kDeqWarpsPerGroup = 4;
-  static constexpr int kDeqGroups = kATmem ? (kAStages < 4 ? kAStages : 4) : (kDeq ? 2 : 0);
+  static constexpr int kDeqGroups = kDeq ? (kAStages < (kATmem ? 4 : 2) ? kAStages : (kATmem ? 4 : 2)) : 0;
   static constexpr int kQWarp = 6 + 4 * kDeqGroups;
   static constexpr int kThreads = kDeq ? 32 * (kQWarp + 1) : 64 + 128;
   static constexpr int kTmemNeed = kAColBase + (kATmem ? kAStages * kAColsStage : 0);
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
     }
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], C::kAbsTma ? 1 : 1 + 32);  // the TMA arrive (+ one cp.async arrive per producer lane)
-      mbar_init(&q_empty[s], C::kDeqWarpsPerGroup);
+      mbar_init(&q_empty[s], C::kDeqWarpsPerGroup * 32);  // every lane of the consuming group
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
@@ -606,8 +607,11 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
               words[6] = c23.z;
               words[7] = c23.w;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&q_empty[qs]);  // the stage is in registers: the slot may refill
+            // the stage is in registers: the slot may refill.  Every lane arrives for itself after a proxy
+            // fence, so its own generic reads of the slot are ordered before the refill's TMA (async-proxy)
+            // writes
+            fence_proxy_async_smem();
+            mbar_arrive(&q_empty[qs]);
           }
           // 64 bf16 values (32 registers) of block p: dequantized codes, or the LoRA rows in the extra stages
           auto block_values = [&](int p, uint32_t (&r)[32]) {
@@ -652,6 +656,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
                 }
               }
             } else {
+              // the block's 16 scaled levels in registers, looked up by byte permutes
               const Nf4RegTable tab = nf4_reg_table(sc[p]);
 #pragma unroll
               for (int w = 0; w < 8; ++w) {
@@ -674,6 +679,9 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          // the MMAs of the slot's previous stage read it through the async proxy; order those reads before
+          // this thread's generic writes
+          if constexpr (!C::kATmem) fence_proxy_async_smem();
           if constexpr (C::kATmem) {
             const uint32_t a_col = tmem_base + t_lane + static_cast<uint32_t>(C::kAColBase + as * C::kAColsStage);
             tmem_st_32x32b_x32(a_col, r);

@@ -117,9 +117,8 @@ struct UmmaCfg {
   static constexpr int kCBytes = 4096 * KB;                       // 128 rows x 64 KB codes
   static constexpr int kSBytes = 512 * KB;                        // 128 rows x KB absmax values
   static constexpr int kQSlot = kDeq ? kCBytes + kSBytes : 0;
-  // the TMEM dequantizers look codes up in a shared-memory table of bf16 level pairs, one copy per lane
-  // (32 KB); the MN-major ones use a per-thread register table (exact, no shared-memory reads)
-  static constexpr int kLutBytes = kATmem ? 256 * 32 * 4 : 0;
+  // the dequantizers look codes up in a shared-memory table of bf16 level pairs, one copy per lane (32 KB)
+  static constexpr int kLutBytes = kDeq ? 256 * 32 * 4 : 0;
   static constexpr int kBarBytes = 1024;
   static constexpr int kBudget = 226 * 1024 - 1024 - kLutBytes - kBarBytes;
 
@@ -134,7 +133,7 @@ struct UmmaCfg {
   // A ring may run: the A ring is never deeper than the B ring (then the B phase a dequantizer waits for is
   // always the next one of its slot -- see the parity note in the kernel).  Deep rings when B tiles are
   // small (token-light layers), 4 stages of 16-32 KB otherwise.
-  static constexpr int kBStagesWant = kDeq ? (BN <= 64 ? 8 : 4) : 8;
+  static constexpr int kBStagesWant = kDeq ? (BN <= 64 ? 8 : (AM == A_DEQ_MN && BN >= 256 ? 3 : 4)) : 8;
   static constexpr int kAStagesWant = kATmem ? kAStagesTmem : (AM == A_DEQ_MN ? (BN >= 256 ? 3 : 4) : 0);
   static constexpr int kQWant = KB == 4 ? 6 : (BN >= 128 ? 10 : 16);
   static constexpr int kBFit = (kBudget - kAStagesWant * kASlot - (kDeq ? kQWant * kQSlot : 0)) / kBSlot;
@@ -145,9 +144,9 @@ struct UmmaCfg {
 
   // Dequantizer groups of 4 warps (one per TMEM lane quarter); group g % kDeqGroups takes stage g.  A warp
   // spends most of a stage waiting on its own instruction latencies, so stage throughput grows with the
-  // number of groups in flight, up to the A ring's depth: 4 in the TMEM kernel, 2 in the MN-major one.
+  // number of groups in flight, up to the A ring's depth: 4 in the TMEM kernel, 3 in the MN-major one.
   static constexpr int kDeqWarpsPerGroup = 4;
-  static constexpr int kDeqGroups = kDeq ? (kAStages < (kATmem ? 4 : 2) ? kAStages : (kATmem ? 4 : 2)) : 0;
+  static constexpr int kDeqGroups = kDeq ? (kAStages < (kATmem ? 4 : 3) ? kAStages : (kATmem ? 4 : 3)) : 0;
   static constexpr int kQWarp = 6 + 4 * kDeqGroups;
   static constexpr int kThreads = kDeq ? 32 * (kQWarp + 1) : 64 + 128;
   static constexpr int kTmemNeed = kAColBase + (kATmem ? kAStages * kAColsStage : 0);
@@ -169,57 +168,6 @@ struct UmmaCfg {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   static_assert((2 * (kBStages + kAStages + kQStages) + 4) * 8 + 8 <= kBarBytes, "barrier area");
 };
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-
-// The 16 levels of one block scaled by its absmax and rounded to bf16 -- exactly the values
-// nf4_dequantize(..., bf16) produces -- held in registers as byte planes for byte-permute lookups:
-// lo[j] holds the low bytes of entries 4j..4j+3, hi[j] their high bytes.
-struct Nf4RegTable {
-  uint32_t lo[4], hi[4];
-};
-
-__device__ __forceinline__ Nf4RegTable nf4_reg_table(float sc) {
-  const float lv[16] = {QLORA_NF4_LEVELS};
-  uint32_t p[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(lv[2 * i], sc), __fmul_rn(lv[2 * i + 1], sc));
-    p[i] = *reinterpret_cast<uint32_t*>(&h);
-  }
-  Nf4RegTable t;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    t.lo[j] = prmt(p[2 * j], p[2 * j + 1], 0x6420u);
-    t.hi[j] = prmt(p[2 * j], p[2 * j + 1], 0x7531u);
-  }
-  return t;
-}
-
-// Eight codes (one 32-bit word: byte j = element 2j in the high nibble, 2j+1 in the low nibble) ->
-// eight bf16 values in element order (four bf16 pairs, first element in the low half).
-// Each nibble v selects byte (v & 7) of the table half v >> 3; a byte mask from bit 3 picks the half.
-__device__ __forceinline__ void nf4_lookup8(const Nf4RegTable& t, uint32_t q, uint32_t (&o)[4]) {
-  const uint32_t s0 = q & 0x77777777u;
-  const uint32_t b0 = (q >> 3) & 0x11111111u;
-  const uint32_t s1 = s0 >> 16;
-  const uint32_t b1 = b0 >> 16;
-  const uint32_t m0 = prmt(0x0000FF00u, 0u, b0);  // byte i: 0xFF when code (i ^ 1) of the low half is >= 8
-  const uint32_t m1 = prmt(0x0000FF00u, 0u, b1);
-  const uint32_t L0 = (prmt(t.lo[0], t.lo[1], s0) & ~m0) | (prmt(t.lo[2], t.lo[3], s0) & m0);
-  const uint32_t H0 = (prmt(t.hi[0], t.hi[1], s0) & ~m0) | (prmt(t.hi[2], t.hi[3], s0) & m0);
-  const uint32_t L1 = (prmt(t.lo[0], t.lo[1], s1) & ~m1) | (prmt(t.lo[2], t.lo[3], s1) & m1);
-  const uint32_t H1 = (prmt(t.hi[0], t.hi[1], s1) & ~m1) | (prmt(t.hi[2], t.hi[3], s1) & m1);
-  // L0/H0 hold elements in the order (1, 0, 3, 2); interleave low and high bytes back into element order
-  o[0] = prmt(L0, H0, 0x4051u);
-  o[1] = prmt(L0, H0, 0x6273u);
-  o[2] = prmt(L1, H1, 0x4051u);
-  o[3] = prmt(L1, H1, 0x6273u);
-}
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, unsigned int* err) {
   const long long t0 = clock64();
@@ -640,7 +588,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
                 r[4 * c + 2] = v.z;
                 r[4 * c + 3] = v.w;
               }
-            } else if constexpr (C::kATmem) {
+            } else {
               // level pair from this lane's copy of the table, times the block scale in bf16x2
               const __nv_bfloat162 sc2 = __float2bfloat162_rn(sc[p]);
 #pragma unroll
@@ -654,18 +602,6 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
                   __nv_bfloat162 pr = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc2);
                   r[4 * w + j] = *reinterpret_cast<uint32_t*>(&pr);
                 }
-              }
-            } else {
-              // the block's 16 scaled levels in registers, looked up by byte permutes
-              const Nf4RegTable tab = nf4_reg_table(sc[p]);
-#pragma unroll
-              for (int w = 0; w < 8; ++w) {
-                uint32_t o[4];
-                nf4_lookup8(tab, words[8 * p + w], o);
-                r[4 * w] = o[0];
-                r[4 * w + 1] = o[1];
-                r[4 * w + 2] = o[2];
-                r[4 * w + 3] = o[3];
               }
             }
           };

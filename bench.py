@@ -43,7 +43,8 @@ def load_peaks() -> dict:
         with open(path) as f:
             p = json.load(f)
         return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
-                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "source": "measured"}
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0)), "source": "measured"}
     except Exception:
         return dict(FALLBACK_PEAKS)
 
@@ -376,6 +377,25 @@ def run_other_workloads(peaks, dev):
                             "dequantize_bf16_ms": round(dq_ms, 4),
                             "dequantize_gbs": round(db / (dq_ms * 1e-3) / 1e9, 1),
                             "dequantize_hbm_frac": round(db / (dq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    del W, codes, absmax
+    # LoRA merge requantized to NF4 in one pass, on the decode layer's weight (28672 x 8192, r = 16).  Its
+    # fixed-order fp32 arithmetic runs on the CUDA cores: 2r + 3 single operations per element (r products,
+    # r additions, the dequantizing product, the scaling, the final addition), against one fp32 operation
+    # per lane per clock (128 lanes per SM).
+    w = I.WORKLOADS["decode_16x8192x28672_r16"]
+    d = I.make_linear_inputs(w)
+    codes, absmax = ops.nf4_quantize(torch.from_numpy(d["W"]).to(dev).reshape(-1))
+    A, B = d["A"].to(dev), d["B"].to(dev)
+    c_out, a_out = torch.empty_like(codes), torch.empty_like(absmax)
+    m_ms = timeit(lambda: ops.merge_lora_nf4(codes, absmax, A, B, w.s, w.N, w.K, codes_out=c_out, absmax_out=a_out))
+    n = w.N * w.K
+    mb = 2 * (n // 2 + n // 64 * 4) + (w.r * w.K + w.N * w.r) * 2
+    alu_ops = n * (2 * w.r + 3)
+    alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * peaks.get("sm_max_mhz", 1965.0) * 1e6
+    res["merge_nf4_28672x8192_r16"] = {"ms": round(m_ms, 4), "gbs": round(mb / (m_ms * 1e-3) / 1e9, 1),
+                                       "hbm_frac": round(mb / (m_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                       "alu_gops": round(alu_ops / (m_ms * 1e-3) / 1e9, 1),
+                                       "alu_frac": round(alu_ops / (m_ms * 1e-3) / alu_peak, 4)}
     return res
 
 

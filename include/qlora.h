@@ -108,6 +108,34 @@ QL_API ql_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64
                          ql_dtype out_dtype, void* out, void* stream);
 
 /*
+ * qlora_merge_lora -- merged weight W' = deq(W) + s * B * A of one layer ("unsloth", pyshine.com, section
+ * "Why You Need This", the paragraph on saving: adapters folded into the base layer by layer).
+ *   N, K     W is [N,K]: N >= 1, K a positive multiple of 64.
+ *   r        LoRA rank, 0 <= r <= 256 (r = 0: W' = deq(W)).
+ *   codes, absmax  the base weight as produced by nf4_quantize (16-byte aligned).
+ *   A        [r,K] bf16 row-major;  B [N,r] bf16 row-major (16-byte aligned; may be null when r = 0).
+ *   s        the LoRA scaling.
+ *   out_dtype QL_F32: out is float[N*K];  QL_BF16: out is bf16[N*K] (round-to-nearest-even of W').
+ * Arithmetic, per element, in IEEE fp32 with no fused multiply-add: d = level * absmax; acc = sum over j
+ * of B[n,j] * A[j,k], added left to right starting from 0; W' = d + s * acc.  Bit-exact and deterministic.
+ * QL_ERR_INVALID_ARG on bad sizes, null or misaligned pointers, or another out_dtype.
+ */
+QL_API ql_status qlora_merge_lora(int64_t N, int64_t K, int64_t r, const uint8_t* codes, const float* absmax,
+                                  const uint16_t* A, const uint16_t* B, float s, ql_dtype out_dtype, void* out,
+                                  void* stream);
+
+/*
+ * qlora_merge_lora_nf4 -- W' as above, requantized in the same pass by the nf4_quantize rule, so the merged
+ * layer stays 4-bit and W' never reaches HBM.
+ *   codes_out  [N*K/2] uint8, absmax_out [N*K/64] fp32 (16-byte aligned).  They may be the input buffers
+ *              themselves (in-place merge): each 64-element block is read in full before it is written.
+ * Bit-exact and deterministic.  A non-finite W' is recorded in the device error word, as in nf4_quantize.
+ */
+QL_API ql_status qlora_merge_lora_nf4(int64_t N, int64_t K, int64_t r, const uint8_t* codes, const float* absmax,
+                                      const uint16_t* A, const uint16_t* B, float s, uint8_t* codes_out,
+                                      float* absmax_out, void* stream);
+
+/*
  * qlora_workspace_bytes -- device scratch needed by qlora_linear_fwd (pass = QL_PASS_FWD) or
  * qlora_linear_bwd (QL_PASS_BWD) for these sizes on the current device (split-K partial sums, the
  * rank-r intermediates s*x*A^T and s*dY*B).  Host-only.  Returns 0 when nothing is needed.

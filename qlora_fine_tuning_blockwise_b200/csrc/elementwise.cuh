@@ -56,6 +56,65 @@ __global__ void nf4_quantize_kernel(const float* __restrict__ w, long long nbloc
   }
 }
 
+// LoRA merge W' = deq(W) + s B A ("unsloth" (pyshine.com), section "Why You Need This": merged saves fold
+// the adapters into the base layer by layer).  One warp per 64-element block of W' (row n of W, columns
+// k0 .. k0 + 63); lane l owns elements 2l, 2l+1.  Every step is one IEEE fp32 operation, never fused, in a
+// fixed order -- d = level * absmax; acc = sum over j of B[n,j] A[j,k], left to right from 0; w' = d + s acc --
+// so that the requantization below is decided on a value any implementation of that order reproduces.
+//   kOut = 0: W' as fp32;  1: W' as bf16 (round-to-nearest-even);  2: W' requantized to NF4 (codes_out,
+//   absmax_out), by the same rule as nf4_quantize_kernel.  In mode 2 the outputs may alias the inputs: a
+//   block is read in full before it is written.
+template <int kOut>
+__global__ void lora_merge_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ absmax,
+                                  const uint16_t* __restrict__ A, const uint16_t* __restrict__ B, float s,
+                                  long long nblocks, int K, int r, void* __restrict__ out, uint8_t* codes_out,
+                                  float* absmax_out, unsigned int* err) {
+  __shared__ float lv[16];
+  if (threadIdx.x < 16) lv[threadIdx.x] = kNF4LevelsDev[threadIdx.x];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int kb = K / 64;
+  const long long warps_total = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long b = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); b < nblocks;
+       b += warps_total) {
+    const long long n = b / kb;
+    const int k0 = static_cast<int>(b % kb) * 64;
+    const uint32_t byte = codes[b * 32 + lane];
+    const float sc = absmax[b];
+    const float d0 = __fmul_rn(lv[byte >> 4], sc);
+    const float d1 = __fmul_rn(lv[byte & 15u], sc);
+    float acc0 = 0.0f, acc1 = 0.0f;
+    const uint16_t* brow = B + n * r;
+    const uint32_t* apair = reinterpret_cast<const uint32_t*>(A + k0) + lane;  // A[j, k0 + 2l .. k0 + 2l + 1]
+    for (int j = 0; j < r; ++j) {
+      const float bj = __uint_as_float(static_cast<uint32_t>(__ldg(brow + j)) << 16);
+      const uint32_t a = __ldg(apair + static_cast<long long>(j) * (K / 2));
+      acc0 = __fadd_rn(acc0, __fmul_rn(bj, __uint_as_float(a << 16)));
+      acc1 = __fadd_rn(acc1, __fmul_rn(bj, __uint_as_float(a & 0xFFFF0000u)));
+    }
+    const float w0 = __fadd_rn(d0, __fmul_rn(s, acc0));
+    const float w1 = __fadd_rn(d1, __fmul_rn(s, acc1));
+    if constexpr (kOut == 0) {
+      reinterpret_cast<float2*>(out)[b * 32 + lane] = make_float2(w0, w1);
+    } else if constexpr (kOut == 1) {
+      reinterpret_cast<__nv_bfloat162*>(out)[b * 32 + lane] = __floats2bfloat162_rn(w0, w1);
+    } else {
+      float m = fmaxf(fabsf(w0), fabsf(w1));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const bool bad = !isfinite(w0) || !isfinite(w1);
+      if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, kDevErrNonFinite);
+      uint32_t c0 = 7, c1 = 7;
+      if (m > 0.0f) {
+        c0 = nf4_code(__fdiv_rn(w0, m));
+        c1 = nf4_code(__fdiv_rn(w1, m));
+      }
+      codes_out[b * 32 + lane] = static_cast<uint8_t>((c0 << 4) | c1);
+      if (lane == 0) absmax_out[b] = m;
+    }
+  }
+}
+
 // Each thread expands 8 elements (4 code bytes) with one absmax.
 template <bool kBf16>
 __global__ void nf4_dequantize_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ absmax,

@@ -387,6 +387,29 @@ ql_status check_linear(int64_t M, int64_t N, int64_t K, int64_t r) {
 }
 
 }  // namespace
+ql_status merge_checks(int64_t N, int64_t K, int64_t r, const uint8_t* codes, const float* absmax, const uint16_t* A,
+                       const uint16_t* B) {
+  if (N < 1 || K < 64 || K % 64 != 0 || r < 0 || r > 256) return QL_ERR_INVALID_ARG;
+  if (N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1) return QL_ERR_INVALID_ARG;
+  if (!codes || !absmax || !aligned16(codes) || !aligned16(absmax)) return QL_ERR_INVALID_ARG;
+  if (r > 0 && (!A || !B || !aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
+  return QL_OK;
+}
+
+template <int kOut>
+ql_status launch_merge(int64_t N, int64_t K, int64_t r, const uint8_t* codes, const float* absmax, const uint16_t* A,
+                       const uint16_t* B, float s, void* out, uint8_t* codes_out, float* absmax_out, void* stream) {
+  DeviceInfo d;
+  if (!device_info(&d)) return QL_ERR_CUDA;
+  const long long nblocks = N * K / 64;
+  const int threads = 256;  // 8 warps = 8 blocks per CTA iteration
+  const long long ctas = std::min<long long>(cdiv(nblocks, 8), static_cast<long long>(d.sms) * 32);
+  lora_merge_kernel<kOut><<<static_cast<unsigned>(ctas), threads, 0, as_stream(stream)>>>(
+      codes, absmax, A, B, s, nblocks, static_cast<int>(K), static_cast<int>(r), out, codes_out, absmax_out, d.err);
+  count_launch();
+  return status_of(cudaGetLastError());
+}
+
 }  // namespace qlora
 
 using namespace qlora;
@@ -638,6 +661,25 @@ ql_status qlora_linear_bwd(int64_t M, int64_t N, int64_t K, int64_t r, const uin
     if (run_gemm(g, dB, false, 1.0f, r, 1, N, r, N * r, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
   }
   return QL_OK;
+}
+
+ql_status qlora_merge_lora(int64_t N, int64_t K, int64_t r, const uint8_t* codes, const float* absmax,
+                           const uint16_t* A, const uint16_t* B, float s, ql_dtype out_dtype, void* out, void* stream) {
+  ql_status st = merge_checks(N, K, r, codes, absmax, A, B);
+  if (st != QL_OK) return st;
+  if (!out || !aligned16(out)) return QL_ERR_INVALID_ARG;
+  if (out_dtype == QL_F32) return launch_merge<0>(N, K, r, codes, absmax, A, B, s, out, nullptr, nullptr, stream);
+  if (out_dtype == QL_BF16) return launch_merge<1>(N, K, r, codes, absmax, A, B, s, out, nullptr, nullptr, stream);
+  return QL_ERR_INVALID_ARG;
+}
+
+ql_status qlora_merge_lora_nf4(int64_t N, int64_t K, int64_t r, const uint8_t* codes, const float* absmax,
+                               const uint16_t* A, const uint16_t* B, float s, uint8_t* codes_out, float* absmax_out,
+                               void* stream) {
+  ql_status st = merge_checks(N, K, r, codes, absmax, A, B);
+  if (st != QL_OK) return st;
+  if (!codes_out || !absmax_out || !aligned16(codes_out) || !aligned16(absmax_out)) return QL_ERR_INVALID_ARG;
+  return launch_merge<2>(N, K, r, codes, absmax, A, B, s, nullptr, codes_out, absmax_out, stream);
 }
 
 ql_status qlora_swiglu_fwd(int64_t numel, const uint16_t* g, const uint16_t* u, uint16_t* h, void* stream) {

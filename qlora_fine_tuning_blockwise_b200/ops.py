@@ -38,6 +38,10 @@ SIGNATURES = {
     "ql_selftest_wait_timeout": (ctypes.c_int, [_c_i64, _c_p]),
     "nf4_quantize": (ctypes.c_int, [_c_p, _c_i64, ctypes.c_int, _c_p, _c_p, _c_p]),
     "nf4_dequantize": (ctypes.c_int, [_c_p, _c_p, _c_i64, ctypes.c_int, ctypes.c_int, _c_p, _c_p]),
+    "qlora_merge_lora": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, ctypes.c_float, ctypes.c_int,
+                                        _c_p, _c_p]),
+    "qlora_merge_lora_nf4": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, ctypes.c_float, _c_p,
+                                            _c_p, _c_p]),
     "qlora_workspace_bytes": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64, _c_i64, ctypes.c_int]),
     "qlora_linear_fwd": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, ctypes.c_float,
                                         _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
@@ -163,6 +167,35 @@ def nf4_dequantize(codes: torch.Tensor, absmax: torch.Tensor, numel: int, blocks
     _check(lib().nf4_dequantize(_ptr(codes), _ptr(absmax), numel, blocksize, code, _ptr(out), _stream(codes.device)),
            "nf4_dequantize")
     return out
+
+
+def merge_lora(codes: torch.Tensor, absmax: torch.Tensor, A, B, s: float, N: int, K: int,
+               dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    """W' = deq(W) + s B A  [N,K] (fp32 or bf16); A [r,K] and B [N,r] bf16, or None for r = 0."""
+    assert codes.is_cuda and codes.dtype == torch.uint8 and absmax.dtype == torch.float32
+    r = 0 if A is None else A.shape[0]
+    out = torch.empty(N, K, dtype=dtype, device=codes.device)
+    code = QL_BF16 if dtype == torch.bfloat16 else QL_F32
+    _check(lib().qlora_merge_lora(N, K, r, _ptr(codes), _ptr(absmax), _ptr(_bits(A) if r else None),
+                                  _ptr(_bits(B) if r else None), float(s), code, _ptr(out), _stream(codes.device)),
+           "qlora_merge_lora")
+    return out
+
+
+def merge_lora_nf4(codes: torch.Tensor, absmax: torch.Tensor, A, B, s: float, N: int, K: int,
+                   codes_out: torch.Tensor | None = None, absmax_out: torch.Tensor | None = None):
+    """(codes', absmax'): W' = deq(W) + s B A requantized to NF4 in one pass.  Passing the input tensors as the
+    outputs merges in place."""
+    assert codes.is_cuda and codes.dtype == torch.uint8 and absmax.dtype == torch.float32
+    r = 0 if A is None else A.shape[0]
+    if codes_out is None:
+        codes_out = torch.empty_like(codes)
+    if absmax_out is None:
+        absmax_out = torch.empty_like(absmax)
+    _check(lib().qlora_merge_lora_nf4(N, K, r, _ptr(codes), _ptr(absmax), _ptr(_bits(A) if r else None),
+                                      _ptr(_bits(B) if r else None), float(s), _ptr(codes_out), _ptr(absmax_out),
+                                      _stream(codes.device)), "qlora_merge_lora_nf4")
+    return codes_out, absmax_out
 
 
 # ------------------------------------------------------------------------------------------ linear layer

@@ -116,3 +116,16 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="not built"):
         ops.lib()
+
+
+def test_merge_rejects_bad_arguments_on_host(L):
+    lib = L.lib()
+    p = ctypes.c_void_p(FAKE)
+    for N, K, r in [(0, 64, 8), (4, 100, 8), (4, 32, 8), (4, 64, -1), (4, 64, 300)]:
+        assert lib.qlora_merge_lora(N, K, r, p, p, p, p, 2.0, 0, p, None) == L.QL_ERR_INVALID_ARG
+        assert lib.qlora_merge_lora_nf4(N, K, r, p, p, p, p, 2.0, p, p, None) == L.QL_ERR_INVALID_ARG
+    assert lib.qlora_merge_lora(4, 64, 8, p, p, None, p, 2.0, 0, p, None) == L.QL_ERR_INVALID_ARG   # A missing
+    assert lib.qlora_merge_lora(4, 64, 8, p, p, p, p, 2.0, 5, p, None) == L.QL_ERR_INVALID_ARG      # bad dtype
+    assert lib.qlora_merge_lora_nf4(4, 64, 8, p, p, p, p, 2.0, None, p, None) == L.QL_ERR_INVALID_ARG
+    assert lib.qlora_merge_lora(4, 64, 8, ctypes.c_void_p(FAKE + 2), p, p, p, 2.0, 0, p, None) == \
+        L.QL_ERR_INVALID_ARG  # misaligned codes

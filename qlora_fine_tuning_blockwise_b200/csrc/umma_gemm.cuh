@@ -27,8 +27,7 @@
 //   A ring:         dequantized A tiles (TMEM columns or shared memory), filled by the dequantizers,
 //                   emptied by the MMAs (tcgen05.commit);
 //   B ring:         B tiles (and A tiles in the TMA modes), filled by the B producer, emptied by the MMAs.
-// In the dequantizing modes the MMA waits on the A ring only: a dequantizer warp arrives there after it has
-// also seen the stage's B tile land.
+// The MMA waits on both the A ring (dequantized tile ready) and the B ring (B tile landed) of each stage.
 //
 // Warp roles: warp 0 = B producer (lane 0 issues TMA), warp 1 = TMEM allocator + MMA issuer, warps 2..5 =
 // epilogue (TMEM -> registers -> global), warps 6 .. 6 + 4G - 1 = dequantizers (G groups of 4 warps; group
@@ -129,16 +128,14 @@ struct UmmaCfg {
   static constexpr int kAColsStage = 32 * KB;
   static constexpr int kAStagesTmem = (512 - kAColBase) / kAColsStage > 8 ? 8 : (512 - kAColBase) / kAColsStage;
 
-  // ring depths.  A dequantizer's arrival waits for the stage's B tile, so the B ring bounds how far ahead the
-  // A ring may run: the A ring is never deeper than the B ring (then the B phase a dequantizer waits for is
-  // always the next one of its slot -- see the parity note in the kernel).  Deep rings when B tiles are
-  // small (token-light layers), 4 stages of 16-32 KB otherwise.
+  // ring depths: deep B rings when B tiles are small (token-light layers), 4 stages of 16-32 KB otherwise;
+  // the A ring as deep as tensor memory (or shared memory, for A_DEQ_MN) allows.
   static constexpr int kBStagesWant = kDeq ? (BN <= 64 ? 8 : (AM == A_DEQ_MN && BN >= 256 ? 3 : 4)) : 8;
   static constexpr int kAStagesWant = kATmem ? kAStagesTmem : (AM == A_DEQ_MN ? (BN >= 256 ? 3 : 4) : 0);
   static constexpr int kQWant = KB == 4 ? 6 : (BN >= 128 ? 10 : 16);
   static constexpr int kBFit = (kBudget - kAStagesWant * kASlot - (kDeq ? kQWant * kQSlot : 0)) / kBSlot;
   static constexpr int kBStages = kBFit < kBStagesWant ? (kBFit < 2 ? 2 : kBFit) : kBStagesWant;
-  static constexpr int kAStages = kAStagesWant > kBStages ? kBStages : kAStagesWant;
+  static constexpr int kAStages = kAStagesWant;
   static constexpr int kQFit = kDeq ? (kBudget - kAStages * kASlot - kBStages * kBSlot) / kQSlot : 0;
   static constexpr int kQStages = kQFit > 16 ? 16 : kQFit;
 
@@ -160,9 +157,9 @@ struct UmmaCfg {
   static_assert(KB == 1 || (kATmem && KB == 4), "4-block stages exist for the TMEM forward only");
   static_assert(kTmemNeed <= 512, "tensor memory");
   static_assert(kBStages >= 2 && (!kDeq || (kAStages >= 2 && kQStages >= 4)), "ring depths");
-  // parity safety (see the kernel): A ring no deeper than the B ring, Q ring deeper than the A ring by at
-  // least the number of dequantizer groups, and no more groups than A slots
-  static_assert(!kDeq || (kAStages <= kBStages && kQStages >= kAStages + kDeqGroups && kDeqGroups <= kAStages),
+  // parity safety (see the kernel): Q ring deeper than the A ring by at least the number of dequantizer
+  // groups, and no more groups than A slots
+  static_assert(!kDeq || (kQStages >= kAStages + kDeqGroups && kDeqGroups <= kAStages),
                 "ring depth relations");
   static_assert(kBStages <= 32 && kAStages <= 32 && kQStages <= 32, "armed-slot bit masks");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -222,8 +219,8 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
   //   - a barrier cannot run ahead: each refill needs the consumer's release of the slot first;
   //   - a dequantizer at stage g has seen the MMAs of stage g - G - AS complete (its own previous stage's
   //     a_empty wait, G = dequantizer groups), so with G <= AS its a_empty wait for stage g - AS cannot see
-  //     an older phase, with QS >= AS + G the Q stage QS before its own has been consumed, and (after the
-  //     a_empty wait) with AS <= BS the B stage BS before its own has landed.
+  //     an older phase, and with QS >= AS + G the Q stage QS before its own has been consumed;
+  //   - the MMA and the producers visit every phase of the barriers they wait on, in order.
   uint64_t* b_full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sLut) + C::kLutBytes);
   uint64_t* b_empty = b_full + BS;
   uint64_t* a_full = b_empty + BS;
@@ -356,9 +353,9 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
         int as = 0;
         bool ok;
         if constexpr (C::kDeq) {
-          // a dequantizer arrives on a_full only after the stage's B tile has landed as well
           as = g % AS;
-          ok = mbar_wait(&a_full[as], static_cast<uint32_t>(g / AS) & 1u, abort_flag, args.err);
+          ok = mbar_wait(&a_full[as], static_cast<uint32_t>(g / AS) & 1u, abort_flag, args.err) &&
+               mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err);
         } else {
           ok = mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err);
         }
@@ -639,10 +636,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
           __syncwarp();
           if (lane == 0) {
             // the MMA waits on a_full alone: arrive only once the stage's B tile has landed as well
-            const int bs = g % BS;
-            bool okb = mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err);
-            if (okb) mbar_arrive(&a_full[as]);
-            else stop = true;
+            mbar_arrive(&a_full[as]);
           }
           stop = __shfl_sync(kFull, stop ? 1 : 0, 0) != 0;
           if (stop) break;

@@ -50,13 +50,19 @@ def load_peaks() -> dict:
 
 
 def kernel_source_sha() -> str:
+    """Hash of the kernel sources' code (comments and whitespace removed): recorded profiler counters stay
+    valid across comment edits and become stale on any code change."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qlora_fine_tuning_blockwise_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+            with open(os.path.join(csrc, name)) as f:
+                text = f.read()
+            text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+            text = re.sub(r"//[^\n]*", " ", text)
+            h.update(name.encode())
+            h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

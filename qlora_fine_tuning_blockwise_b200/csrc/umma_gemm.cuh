@@ -1,7 +1,8 @@
 // tcgen05 GEMM kernel for the QLoRA layer (sm_100a), persistent over work units.
 //
 // A work unit is a 128 x BN fp32 tile of D[i, j] = sum_kk Aop[i, kk] * Bop[j, kk] accumulated in TMEM over
-// one split of the contraction (64-element stages), optionally preceded by "extra" stages that append the
+// one split of the contraction (stages of KB blocks of 64 elements), optionally preceded by "extra" stages
+// that append the
 // rank-r LoRA columns to the contraction ([x | s u] . [deq(W) | B]^T in the forward, [dY | v] . [deq(W); A]
 // in the backward), so base and LoRA products land in one accumulator.  Each CTA walks units
 // blockIdx.x, blockIdx.x + gridDim.x, ...; its rings run on across units, and where tensor memory allows
@@ -10,7 +11,7 @@
 // The weight is always the 128-row (M-side) operand: the kernel computes the transposed product
 // (y^T = deq(W) x^T, dX^T = deq(W)^T dY^T), so one dequantized weight element feeds BN tokens.
 //
-// Operand A, per stage (128 rows x 64 contraction elements, bf16):
+// Operand A, per 64-element block (128 rows x 64 contraction elements, bf16):
 //   A_TMA_K / A_TMA_MN   loaded by TMA from a bf16 matrix (K-major or MN-major) together with B,
 //   A_DEQ_MN             backward: dequantized from NF4 codes into the MN-major 128B-swizzled shared-memory
 //                        layout (rows = W columns k, contraction over W rows n) -- the transpose of deq(W)
@@ -18,12 +19,14 @@
 //   A_DEQ_TMEM           forward: dequantized rows go from registers straight into tensor memory
 //                        (tcgen05.st) and the MMA reads A there, so A never touches shared memory; the
 //                        LoRA stages copy rows of B the same way.
-// Operand B (BN x 64): always by TMA.
+// The dequantizers expand a code byte (two elements) through a lane-replicated shared table of bf16 level
+// pairs and multiply by the block scale in bf16x2.
+// Operand B (BN x 64 per block): always by TMA.
 //
 // Three rings decouple the latencies of the dequantizing kernels:
-//   Q ring (deep):  packed codes (TMA) + the stage's 128 absmax values (cp.async), filled by the Q producer
-//                   as far ahead as its depth allows, emptied as soon as a dequantizer has the stage in
-//                   registers -- so HBM latency overlaps many stages of work;
+//   Q ring (deep):  packed codes (TMA) + the stage's absmax values (one cp.async per row, or one TMA box in
+//                   4-block stages), filled by the Q producer as far ahead as its depth allows, emptied as
+//                   soon as a dequantizer has the stage in registers -- so HBM latency overlaps many stages;
 //   A ring:         dequantized A tiles (TMEM columns or shared memory), filled by the dequantizers,
 //                   emptied by the MMAs (tcgen05.commit);
 //   B ring:         B tiles (and A tiles in the TMA modes), filled by the B producer, emptied by the MMAs.
@@ -36,7 +39,9 @@
 //
 // Shared-memory tiles: for the 128B swizzle every tile starts on a 1024-byte boundary; row r of a tile is
 // 128 bytes at r*128 and its 16-byte chunk c sits at chunk position c ^ (r & 7).  TMA writes that layout;
-// the dequantizers write it with plain 16-byte stores followed by fence.proxy.async.
+// the dequantizers write it with plain 16-byte stores.  Slots change hands between the generic proxy
+// (thread loads and stores) and the async proxy (TMA, MMA), so each handoff carries a fence.proxy.async:
+// before a codes slot is released for a TMA refill, and before an A slot the MMAs read is overwritten.
 //
 // Every wait is bounded; on expiry the waiting thread raises the CTA's abort flag and the device error word,
 // every role leaves its loop, and the producers wait (bounded) for their copies in flight before the CTA
@@ -56,7 +61,7 @@ struct UmmaArgs {
   int rows, cols;         // D extent: i in [0, rows), j in [0, cols)
   int tiles_i, tiles_j;   // ceil(rows / 128), ceil(cols / BN)
   int splits;             // contraction splits; units = splits * tiles_i * tiles_j
-  int k_stages;           // main contraction stages (64 elements each) in total
+  int k_stages;           // main contraction stages (64 KB elements each) in total
   int stages_per_split;   // main stages per split
   int n_extra;            // extra (LoRA) stages, run by split 0 only, before its main stages
   // dequantization (A_DEQ_*): W is [w_rows, w_cols] with absmax [w_rows, w_cols / 64]

@@ -276,52 +276,95 @@ def run_ours(args, rank, world, local, peaks):
 
 
 def run_e2e(ctx, args, world):
-    """Same metric through the public API with host buffers: pinned H2D of x and dY, D2H of y, dX, dA, dB."""
+    """Same metric through the public API with host buffers: every step copies its x and dY in from pinned host
+    memory and its y, dX, dA, dB out to pinned host memory.  Steps are pipelined over three streams -- the
+    host-to-device copies of step i + 1 and the device-to-host copies of step i - 1 run while step i computes --
+    with double-buffered device inputs and outputs, ordered by events.  The L2 flush runs on the compute stream
+    at the start of every step, inside the timed interval.  Time = device time from the first copy in to the
+    last copy out, max over ranks."""
     import torch
     import torch.distributed as dist
 
+    from qlora_fine_tuning_blockwise_b200 import ops
     from qlora_fine_tuning_blockwise_b200.parallel import allreduce_adapter_grads
 
-    layer, x_dev, dy_dev, d, w, dev = ctx
+    layer, _x_dev, _dy_dev, d, w, dev = ctx
     x_h = d["x"].pin_memory()
     dy_h = d["dy"].pin_memory()
-    outs_h = None
-    stream = torch.cuda.current_stream(dev)
+    M, N, K, r = w.M, w.N, w.K, w.r
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    bufs = layer._buffers(M, dev)  # workspaces: used by the compute stream only, in order
+    slots = []
+    for _ in range(2):
+        slots.append(dict(
+            x=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
+            dy=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+            y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+            su=torch.empty(M, r, dtype=torch.bfloat16, device=dev) if r else None,
+            dx=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
+            dA=torch.empty(r, K, dtype=torch.float32, device=dev) if r else None,
+            dB=torch.empty(N, r, dtype=torch.float32, device=dev) if r else None,
+            h=[torch.empty(shape, dtype=dt, pin_memory=True)
+               for shape, dt in (((M, N), torch.bfloat16), ((M, K), torch.bfloat16),
+                                 ((max(r, 1), K), torch.float32), ((N, max(r, 1)), torch.float32))],
+            in_ready=torch.cuda.Event(), computed=torch.cuda.Event(), out_done=torch.cuda.Event()))
+    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def step():
-        nonlocal outs_h
-        x = x_h.to(dev, non_blocking=True)
-        dy = dy_h.to(dev, non_blocking=True)
-        y, su = layer.forward(x)
-        dx, dA, dB = layer.backward(dy, x, su=su)
-        if world > 1:
-            allreduce_adapter_grads([dA, dB])
-        if outs_h is None:
-            outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (y, dx, dA, dB)]
-        for h, t in zip(outs_h, (y, dx, dA, dB)):
-            h.copy_(t, non_blocking=True)
-        return outs_h
+    def issue(i):
+        sl = slots[i % 2]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(sl["computed"])  # step i - 2 has finished reading this slot's inputs
+            sl["x"].copy_(x_h, non_blocking=True)
+            sl["dy"].copy_(dy_h, non_blocking=True)
+            sl["in_ready"].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(sl["in_ready"])
+            if i >= 2:
+                s_comp.wait_event(sl["out_done"])  # step i - 2's outputs have left this slot
+            flush_l2(flush)
+            ops.qlora_linear_fwd(sl["x"], layer.codes, layer.absmax, layer.A, layer.B, layer.s, N, K,
+                                 workspace=bufs["ws_f"], y=sl["y"], su=sl["su"])
+            ops.qlora_linear_bwd(sl["dy"], sl["x"], layer.codes, layer.absmax, layer.A, layer.B, layer.s, N, K,
+                                 su=sl["su"], workspace=bufs["ws_b"], dx=sl["dx"], dA=sl["dA"], dB=sl["dB"])
+            if world > 1:
+                allreduce_adapter_grads([sl["dA"], sl["dB"]])
+            sl["computed"].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(sl["computed"])
+            outs = [t for t in (sl["y"], sl["dx"], sl["dA"], sl["dB"]) if t is not None]
+            for hbuf, t in zip(sl["h"], outs):
+                hbuf.view(-1)[: t.numel()].copy_(t.view(-1), non_blocking=True)
+            sl["out_done"].record(s_out)
+        return outs
 
-    for _ in range(max(args.warmup, 3)):
-        step()
+    for i in range(max(args.warmup, 3)):
+        issue(i)
     torch.cuda.synchronize(dev)
-    K = args.steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    K_steps = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
-    for i in range(K):
-        flush_l2(flush)
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    total = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
-    h2d = x_h.numel() * 2 + dy_h.numel() * 2
-    d2h = sum(t.numel() * t.element_size() for t in outs_h)
-    val = (w.flops_fwd + w.flops_bwd) * world * K / (total * 1e-3) / 1e12
+    start.record(s_in)
+    outs = None
+    for i in range(K_steps):
+        outs = issue(i)
+    # every stream's work is done before the end mark
+    for st in (s_in, s_comp):
+        ev = torch.cuda.Event()
+        ev.record(st)
+        s_out.wait_event(ev)
+    end.record(s_out)
+    torch.cuda.synchronize(dev)
+    total = max_over_ranks(start.elapsed_time(end), world)
+    h2d = (M * K + M * N) * 2
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    val = (w.flops_fwd + w.flops_bwd) * world * K_steps / (total * 1e-3) / 1e12
     return {"value": round(val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": round(total / K, 4)}
+            "ms_per_step": round(total / K_steps, 4),
+            "pipelining": "three streams: copies in of step i+1 and out of step i-1 overlap step i; L2 flushed at the "
+                          "start of every step's compute (inside the timed interval)"}
 
 
 def run_other_workloads(peaks, dev):

@@ -1,0 +1,51 @@
+"""Host-side checks of the benchmark's bookkeeping (no GPU): the kernel-source hash that keys recorded profiler
+counters ignores comments but not code, and recorded DRAM traffic is reported only for the code it was taken on."""
+
+import importlib.util
+import json
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def load_bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    b = load_bench()
+    csrc = tmp_path / "qlora_fine_tuning_blockwise_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cuh").write_text("int f(int a) {\n  return a + 1;  // one\n}\n/* block */\n")
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    h0 = b.kernel_source_sha()
+    (csrc / "k.cuh").write_text("// a new header comment\nint f(int a) {\n    return a + 1;   // changed comment\n}\n")
+    assert b.kernel_source_sha() == h0
+    (csrc / "k.cuh").write_text("int f(int a) {\n  return a + 2;\n}\n")
+    assert b.kernel_source_sha() != h0
+
+
+def test_recorded_traffic_only_for_matching_code(tmp_path, monkeypatch):
+    b = load_bench()
+    csrc = tmp_path / "qlora_fine_tuning_blockwise_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("int main() { return 0; }\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    rec = {"source_sha": b.kernel_source_sha(), "kernels": {"fused_dx": 123}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert b.load_traffic() == {"fused_dx": 123}
+    (csrc / "k.cu").write_text("int main() { return 1; }\n")
+    assert b.load_traffic() == {}
+
+
+def test_committed_traffic_matches_the_committed_kernels():
+    """profiles/traffic.json is keyed to the kernel sources in this tree, so the bench reports it."""
+    b = load_bench()
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    assert rec["source_sha"] == b.kernel_source_sha()
+    assert set(rec["kernels"]) == {"fused_fwd", "fused_dx"} and all(v > 0 for v in rec["kernels"].values())

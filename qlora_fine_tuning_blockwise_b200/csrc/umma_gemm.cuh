@@ -639,7 +639,9 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
             fence_proxy_async_smem();
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(&a_full[as]);  // the warp's quarter of the A stage is in place
+          if (lane == 0) {
+            mbar_arrive(&a_full[as]);  // the warp's quarter of the A stage is in place
+          }
           stop = __shfl_sync(kFull, stop ? 1 : 0, 0) != 0;
           if (stop) break;
         }

@@ -10,6 +10,7 @@ Modules
 ``oracle.nf4``     NF4 codebook, blockwise quantize / dequantize, bf16 round-to-nearest-even.
 ``oracle.linear``  forward / backward of the QLoRA linear layer, SwiGLU, and the gated-MLP chain.
 ``oracle.merge``   LoRA merge W' = deq(W) + s B A and its NF4 requantization.
+``oracle.double_quant``  double quantization of the block constants (8-bit E4M3 codes, 256 per group).
 
 Pins: every function here is checked by ``tests/test_oracle_*.py`` against values fixed by the
 mathematics (closed forms, invariants, brute force on tiny inputs, finite differences, library routines
@@ -18,4 +19,4 @@ the pages name the level set but print no table ("parity unpinned" against the p
 values; see ``oracle.nf4.nf4_codebook``).
 """
 
-from . import nf4, linear, merge  # noqa: F401
+from . import nf4, linear, merge, double_quant  # noqa: F401

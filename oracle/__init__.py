@@ -11,6 +11,7 @@ Modules
 ``oracle.linear``  forward / backward of the QLoRA linear layer, SwiGLU, and the gated-MLP chain.
 ``oracle.merge``   LoRA merge W' = deq(W) + s B A and its NF4 requantization.
 ``oracle.double_quant``  double quantization of the block constants (8-bit E4M3 codes, 256 per group).
+``oracle.nvfp4``   the NVFP4 base-weight format: E2M1 codes, an E4M3 scale per 16, one fp32 scale per tensor.
 
 Pins: every function here is checked by ``tests/test_oracle_*.py`` against values fixed by the
 mathematics (closed forms, invariants, brute force on tiny inputs, finite differences, library routines
@@ -19,4 +20,4 @@ the pages name the level set but print no table ("parity unpinned" against the p
 values; see ``oracle.nf4.nf4_codebook``).
 """
 
-from . import nf4, linear, merge, double_quant  # noqa: F401
+from . import nf4, linear, merge, double_quant, nvfp4  # noqa: F401

@@ -49,13 +49,19 @@ def load_peaks() -> dict:
         return dict(FALLBACK_PEAKS)
 
 
+# The sources of the layer library (libqlora's qlora.cu translation unit and what it includes): the kernels
+# whose counters are recorded under profiles/ are built from these and nothing else.  The format conversions
+# (formats.cu, formats.cuh) are a separate translation unit that none of them includes.
+LAYER_SOURCES = ("elementwise.cuh", "nf4_table.cuh", "ptx.cuh", "qlora.cu", "umma_gemm.cuh")
+
+
 def kernel_source_sha() -> str:
-    """Hash of the kernel sources' code (comments and whitespace removed): recorded profiler counters stay
-    valid across comment edits and become stale on any code change."""
+    """Hash of the layer kernels' source code (comments and whitespace removed): recorded profiler counters
+    stay valid across comment edits and become stale on any code change."""
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qlora_fine_tuning_blockwise_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(LAYER_SOURCES):
         if name.endswith((".cu", ".cuh")):
             with open(os.path.join(csrc, name)) as f:
                 text = f.read()

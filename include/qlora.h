@@ -233,6 +233,73 @@ QL_API ql_status qlora_swiglu_gated_fwd(int64_t M, int64_t F, const uint16_t* gu
 QL_API ql_status qlora_swiglu_gated_bwd(int64_t M, int64_t F, const uint16_t* dh, const uint16_t* gu,
                                         uint16_t* dgu, void* stream);
 
+/* ------------------------------------------------------------------------------------------------------
+ * Weight-format conversions (their own translation unit; their own launch counter and device error word).
+ * ------------------------------------------------------------------------------------------------------ */
+
+/* Number of format-conversion kernels launched in the process so far (all devices).  Host-only. */
+QL_API uint64_t ql_formats_launch_count(void);
+
+/* Reads and clears the format conversions' device error word after synchronizing `stream`.  Returns
+ * QL_ERR_INVALID_ARG if a conversion met a non-finite input (or a negative block constant, or a NaN code),
+ * QL_OK otherwise, or QL_ERR_CUDA.  Synchronizes. */
+QL_API ql_status ql_formats_get_device_error(void* stream);
+
+/*
+ * nf4_double_quantize -- double quantization of the NF4 block constants ("Unsloth v0.1.463-beta: Fixes
+ * Studio Crash and llama-server Permission Issue", kongchang.com, section "About the Unsloth Project",
+ * paragraph "How LoRA and QLoRA work": QLoRA quantizes its quantization constants a second time).
+ *   absmax   [nb] fp32, the block constants as nf4_quantize writes them (finite, >= 0), nb >= 1.
+ *   code8    [nb] uint8 out: per constant, the E4M3 bit pattern of the level nearest to n = fl32(d / c1),
+ *            d = fl32(absmax - mu); the levels are the finite E4M3 values / 448 rounded to fp32; a tie
+ *            goes to the lower level; c1 = 0 gives code 0x00.
+ *   c1       [ceil(nb / 256)] fp32 out: per group of 256 consecutive constants (the last may be shorter),
+ *            max |d| over the group.
+ *   mu       [1] fp32 out (device): the mean of all constants, summed in fp64 group by group in index
+ *            order, the group sums added in order, divided by nb in fp64, rounded to fp32.
+ *   scratch  device scratch of at least nf4_double_quantize_scratch_bytes(nb) bytes (the group sums).
+ * Dequantized by nf4_double_dequantize.  Storage: about 0.127 bit per weight instead of 0.5.  Bit-exact and
+ * deterministic.  All pointers 16-byte aligned.  QL_ERR_INVALID_ARG on bad sizes, null or misaligned
+ * pointers, or too little scratch.  A non-finite or negative constant is recorded in the format device
+ * error word.  The mean is one sequential fp64 sum over the groups: a one-time conversion.
+ */
+QL_API size_t nf4_double_quantize_scratch_bytes(int64_t nb);
+QL_API ql_status nf4_double_quantize(const float* absmax, int64_t nb, uint8_t* code8, float* c1, float* mu,
+                                     void* scratch, size_t scratch_bytes, void* stream);
+
+/*
+ * nf4_double_dequantize -- absmax'[i] = fl32(fl32(L[code8[i]] * c1[i / 256]) + mu), fp32 [nb], from the
+ * outputs of nf4_double_quantize (mu a device pointer).  A NaN code (0x7F, 0xFF) gives NaN and is recorded
+ * in the format device error word.  Bit-exact.  Pointers 16-byte aligned.
+ */
+QL_API ql_status nf4_double_dequantize(const uint8_t* code8, const float* c1, const float* mu, int64_t nb,
+                                       float* absmax_out, void* stream);
+
+/*
+ * nvfp4_quantize -- NVFP4 quantization of a weight ("Major Unsloth Update: NVFP4 Quantization Export and
+ * DeepSeek-V4 Training Support", kongchang.com, section "NVFP4: A Quantization Format for the Next
+ * Generation of Hardware": E2M1 values with a range of about +-6, one FP8 scale per small group).
+ *   w            [numel] fp32, flat row-major; numel a positive multiple of 16 (blocks never straddle rows
+ *                when the row length is a multiple of 16).
+ *   codes        [numel / 2] uint8 out: E2M1 patterns, element 2j in the LOW nibble of byte j.
+ *   scales       [numel / 16] uint8 out: E4M3 pattern of each block's scale.
+ *   tensor_scale [1] fp32 out (device): S = fl32(amax / 2688), amax = max |w| (0 for an all-zero tensor).
+ * Per block of 16 with largest magnitude a: t = fl32(a / fl32(6 S)); scale = E4M3 of t (nearest, ties to
+ * even, saturating at 448); D = fl32(value(scale) * S); code = E2M1 of fl32(w / D) (nearest, ties to the
+ * even mantissa, saturating at 6, sign kept), or +0 when D = 0.  Bit-exact and deterministic.  Pointers
+ * 16-byte aligned.  A non-finite weight is recorded in the format device error word.
+ */
+QL_API ql_status nvfp4_quantize(const float* w, int64_t numel, uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                void* stream);
+
+/*
+ * nvfp4_dequantize -- w' = fl32(value(code) * D), D = fl32(value(scale) * S), from the outputs of
+ * nvfp4_quantize.  out_dtype QL_F32: out is float[numel]; QL_BF16: bf16[numel], round-to-nearest-even of
+ * w'.  Bit-exact.  Pointers 16-byte aligned.
+ */
+QL_API ql_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                                  int64_t numel, ql_dtype out_dtype, void* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -17,8 +17,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqlora.so")
-SOURCES = [os.path.join(CSRC, "qlora.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "umma_gemm.cuh", "elementwise.cuh", "nf4_table.cuh")] + [
+SOURCES = [os.path.join(CSRC, "qlora.cu"), os.path.join(CSRC, "formats.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "umma_gemm.cuh", "elementwise.cuh", "nf4_table.cuh", "formats.cuh")] + [
     os.path.join(ROOT, "include", "qlora.h")
 ]
 

@@ -53,6 +53,13 @@ SIGNATURES = {
     "qlora_swiglu_bwd": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
     "qlora_swiglu_gated_fwd": (ctypes.c_int, [_c_i64, _c_i64, _c_p, _c_p, _c_p]),
     "qlora_swiglu_gated_bwd": (ctypes.c_int, [_c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
+    "ql_formats_launch_count": (ctypes.c_uint64, []),
+    "ql_formats_get_device_error": (ctypes.c_int, [_c_p]),
+    "nf4_double_quantize_scratch_bytes": (ctypes.c_size_t, [_c_i64]),
+    "nf4_double_quantize": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
+    "nf4_double_dequantize": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i64, _c_p, _c_p]),
+    "nvfp4_quantize": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_p, _c_p, _c_p]),
+    "nvfp4_dequantize": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i64, ctypes.c_int, _c_p, _c_p]),
 }
 
 
@@ -196,6 +203,63 @@ def merge_lora_nf4(codes: torch.Tensor, absmax: torch.Tensor, A, B, s: float, N:
                                       _ptr(_bits(B) if r else None), float(s), _ptr(codes_out), _ptr(absmax_out),
                                       _stream(codes.device)), "qlora_merge_lora_nf4")
     return codes_out, absmax_out
+
+
+# ------------------------------------------------------------------------------------------ weight formats
+
+
+def formats_device_error(device: torch.device | None = None) -> int:
+    """Status from the format conversions' device error word (synchronizes the current stream)."""
+    return int(lib().ql_formats_get_device_error(_stream(device)))
+
+
+def formats_launch_count() -> int:
+    """Format-conversion kernels this library has launched in this process."""
+    return int(lib().ql_formats_launch_count())
+
+
+def nf4_double_quantize(absmax: torch.Tensor):
+    """Double quantization of the NF4 block constants: (code8 uint8 [nb], c1 fp32 [ceil(nb/256)], mu fp32 [1])."""
+    assert absmax.is_cuda and absmax.dtype == torch.float32 and absmax.is_contiguous()
+    nb = absmax.numel()
+    code8 = torch.empty(nb, dtype=torch.uint8, device=absmax.device)
+    c1 = torch.empty((nb + 255) // 256, dtype=torch.float32, device=absmax.device)
+    mu = torch.empty(1, dtype=torch.float32, device=absmax.device)
+    need = int(lib().nf4_double_quantize_scratch_bytes(nb))
+    scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=absmax.device)
+    _check(lib().nf4_double_quantize(_ptr(absmax), nb, _ptr(code8), _ptr(c1), _ptr(mu), _ptr(scratch), need,
+                                     _stream(absmax.device)), "nf4_double_quantize")
+    return code8, c1, mu
+
+
+def nf4_double_dequantize(code8: torch.Tensor, c1: torch.Tensor, mu: torch.Tensor) -> torch.Tensor:
+    """absmax' fp32 [nb] from the outputs of nf4_double_quantize."""
+    assert code8.is_cuda and code8.dtype == torch.uint8 and c1.dtype == torch.float32 and mu.dtype == torch.float32
+    out = torch.empty(code8.numel(), dtype=torch.float32, device=code8.device)
+    _check(lib().nf4_double_dequantize(_ptr(code8), _ptr(c1), _ptr(mu), code8.numel(), _ptr(out),
+                                       _stream(code8.device)), "nf4_double_dequantize")
+    return out
+
+
+def nvfp4_quantize(w: torch.Tensor):
+    """w: CUDA fp32 contiguous -> (codes uint8 [numel/2], scales uint8 [numel/16] (E4M3), S fp32 [1])."""
+    assert w.is_cuda and w.dtype == torch.float32 and w.is_contiguous()
+    n = w.numel()
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(n // 16, dtype=torch.uint8, device=w.device)
+    S = torch.empty(1, dtype=torch.float32, device=w.device)
+    _check(lib().nvfp4_quantize(_ptr(w), n, _ptr(codes), _ptr(scales), _ptr(S), _stream(w.device)), "nvfp4_quantize")
+    return codes, scales, S
+
+
+def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, S: torch.Tensor, numel: int,
+                     dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    assert codes.is_cuda and codes.dtype == torch.uint8 and scales.dtype == torch.uint8 and S.dtype == torch.float32
+    out = torch.empty(numel, dtype=dtype, device=codes.device)
+    code = QL_BF16 if dtype == torch.bfloat16 else QL_F32
+    _check(lib().nvfp4_dequantize(_ptr(codes), _ptr(scales), _ptr(S), numel, code, _ptr(out), _stream(codes.device)),
+           "nvfp4_dequantize")
+    return out
 
 
 # ------------------------------------------------------------------------------------------ linear layer

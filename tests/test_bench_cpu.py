@@ -23,6 +23,7 @@ def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     csrc.mkdir(parents=True)
     (csrc / "k.cuh").write_text("int f(int a) {\n  return a + 1;  // one\n}\n/* block */\n")
     monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    monkeypatch.setattr(b, "LAYER_SOURCES", ("k.cuh",))
     h0 = b.kernel_source_sha()
     (csrc / "k.cuh").write_text("// a new header comment\nint f(int a) {\n    return a + 1;   // changed comment\n}\n")
     assert b.kernel_source_sha() == h0
@@ -37,11 +38,30 @@ def test_recorded_traffic_only_for_matching_code(tmp_path, monkeypatch):
     (csrc / "k.cu").write_text("int main() { return 0; }\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    monkeypatch.setattr(b, "LAYER_SOURCES", ("k.cu",))
     rec = {"source_sha": b.kernel_source_sha(), "kernels": {"fused_dx": 123}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     assert b.load_traffic() == {"fused_dx": 123}
     (csrc / "k.cu").write_text("int main() { return 1; }\n")
     assert b.load_traffic() == {}
+
+
+def test_hashed_sources_are_the_layer_translation_unit():
+    """The hash covers exactly qlora.cu and the files it includes (transitively), and no other source: the
+    format conversions (a translation unit of their own) do not make the layer kernels' counters stale."""
+    import re
+    b = load_bench()
+    csrc = os.path.join(ROOT, "qlora_fine_tuning_blockwise_b200", "csrc")
+    seen, todo = set(), ["qlora.cu"]
+    while todo:
+        name = todo.pop()
+        if name in seen:
+            continue
+        seen.add(name)
+        text = open(os.path.join(csrc, name)).read()
+        todo += [m for m in re.findall(r'#include\s+"([^"/]+)"', text) if os.path.exists(os.path.join(csrc, m))]
+    assert seen == set(b.LAYER_SOURCES)
+    assert "formats.cu" not in seen and "formats.cuh" not in seen
 
 
 def test_committed_traffic_record():

@@ -281,13 +281,23 @@ def run_ours(args, rank, world, local, peaks):
     return out, (layer, x, dy, d, w, dev)
 
 
-def run_e2e(ctx, args, world):
+E2E_RESULTS = {
+    # the step's result read back to the host: the adapter gradients, which are what a training step of this
+    # layer produces (y and dX are activations that the neighbouring layers consume on the device)
+    "grads": ("dA", "dB"),
+    # every output of the step
+    "all": ("y", "dx", "dA", "dB"),
+}
+
+
+def run_e2e(ctx, args, world, read_back: str = "grads"):
     """Same metric through the public API with host buffers: every step copies its x and dY in from pinned host
-    memory and its y, dX, dA, dB out to pinned host memory.  Steps are pipelined over three streams -- the
-    host-to-device copies of step i + 1 and the device-to-host copies of step i - 1 run while step i computes --
-    with double-buffered device inputs and outputs, ordered by events.  The L2 flush runs on the compute stream
-    at the start of every step, inside the timed interval.  Time = device time from the first copy in to the
-    last copy out, max over ranks."""
+    memory and its result out to pinned host memory (``E2E_RESULTS[read_back]``).  Steps are pipelined over three
+    streams -- the host-to-device copies of step i + 1 and the device-to-host copies of step i - 1 run while
+    step i computes -- with double-buffered device inputs and outputs, ordered by events.  Every step computes
+    the whole forward and backward whatever is read back.  The L2 flush runs on the compute stream at the start
+    of every step, inside the timed interval.  Time = device time from the first copy in to the last copy out,
+    max over ranks."""
     import torch
     import torch.distributed as dist
 
@@ -310,9 +320,9 @@ def run_e2e(ctx, args, world):
             dx=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
             dA=torch.empty(r, K, dtype=torch.float32, device=dev) if r else None,
             dB=torch.empty(N, r, dtype=torch.float32, device=dev) if r else None,
-            h=[torch.empty(shape, dtype=dt, pin_memory=True)
-               for shape, dt in (((M, N), torch.bfloat16), ((M, K), torch.bfloat16),
-                                 ((max(r, 1), K), torch.float32), ((N, max(r, 1)), torch.float32))],
+            h={name: torch.empty(shape, dtype=dt, pin_memory=True)
+               for name, shape, dt in (("y", (M, N), torch.bfloat16), ("dx", (M, K), torch.bfloat16),
+                                       ("dA", (max(r, 1), K), torch.float32), ("dB", (N, max(r, 1)), torch.float32))},
             in_ready=torch.cuda.Event(), computed=torch.cuda.Event(), out_done=torch.cuda.Event()))
     s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
@@ -338,9 +348,10 @@ def run_e2e(ctx, args, world):
             sl["computed"].record(s_comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(sl["computed"])
-            outs = [t for t in (sl["y"], sl["dx"], sl["dA"], sl["dB"]) if t is not None]
-            for hbuf, t in zip(sl["h"], outs):
-                hbuf.view(-1)[: t.numel()].copy_(t.view(-1), non_blocking=True)
+            names = [nm for nm in E2E_RESULTS[read_back] if sl[nm] is not None] or ["dx"]  # r = 0: no gradients
+            outs = [sl[nm] for nm in names]
+            for nm, t in zip(names, outs):
+                sl["h"][nm].view(-1)[: t.numel()].copy_(t.view(-1), non_blocking=True)
             sl["out_done"].record(s_out)
         return outs
 
@@ -368,7 +379,7 @@ def run_e2e(ctx, args, world):
     d2h = sum(t.numel() * t.element_size() for t in outs)
     val = (w.flops_fwd + w.flops_bwd) * world * K_steps / (total * 1e-3) / 1e12
     return {"value": round(val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": round(total / K_steps, 4),
+            "ms_per_step": round(total / K_steps, 4), "read_back": "+".join(E2E_RESULTS[read_back]),
             "pipelining": "three streams: copies in of step i+1 and out of step i-1 overlap step i; L2 flushed at the "
                           "start of every step's compute (inside the timed interval)"}
 
@@ -562,7 +573,9 @@ def main():
     peaks = load_peaks()
     rank, world, local = dist_setup(args.gpus)
     out, ctx = run_ours(args, rank, world, local, peaks)
-    out["e2e"] = run_e2e(ctx, args, world)
+    out["e2e"] = run_e2e(ctx, args, world, "grads")
+    full = run_e2e(ctx, args, world, "all")
+    out["e2e"]["all_outputs"] = {k: full[k] for k in ("value", "ms_per_step", "d2h_bytes_per_step", "read_back")}
     if rank == 0 and world == 1:
         import torch
         if not args.only_main:

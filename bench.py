@@ -462,6 +462,31 @@ def run_other_workloads(peaks, dev):
                                        "hbm_frac": round(mb / (m_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                                        "alu_gops": round(alu_ops / (m_ms * 1e-3) / 1e9, 1),
                                        "alu_frac": round(alu_ops / (m_ms * 1e-3) / alu_peak, 4)}
+    # Weight-format conversions on the same weight: NVFP4 quantize / dequantize (bf16) and the double
+    # quantization of its NF4 block constants.  Kept apart so that a failure here cannot lose the line.
+    try:
+        Wd = torch.from_numpy(d["W"]).to(dev).reshape(-1)
+        nb = absmax.numel()
+        fq_ms = timeit(lambda: ops.nvfp4_quantize(Wd))
+        fc, fs, fS = ops.nvfp4_quantize(Wd)
+        fd_ms = timeit(lambda: ops.nvfp4_dequantize(fc, fs, fS, n, dtype=torch.bfloat16))
+        dq_ms = timeit(lambda: ops.nf4_double_quantize(absmax))
+        q8, c1, mu = ops.nf4_double_quantize(absmax)
+        dd_ms = timeit(lambda: ops.nf4_double_dequantize(q8, c1, mu))
+        fqb = 2 * n * 4 + n // 2 + n // 16     # the weight read twice (largest magnitude, then blocks)
+        fdb = n // 2 + n // 16 + n * 2
+        dqb = 2 * nb * 4 + nb + (nb + 255) // 256 * (4 + 2 * 8)
+        ddb = nb + (nb + 255) // 256 * 4 + nb * 4
+
+        def hbm(b, ms):
+            return {"ms": round(ms, 4), "gbs": round(b / (ms * 1e-3) / 1e9, 1),
+                    "hbm_frac": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+        res["formats_28672x8192"] = {"nvfp4_quantize": hbm(fqb, fq_ms), "nvfp4_dequantize_bf16": hbm(fdb, fd_ms),
+                                     "nf4_double_quantize": hbm(dqb, dq_ms),
+                                     "nf4_double_dequantize": hbm(ddb, dd_ms)}
+        del Wd, fc, fs, fS, q8, c1, mu
+    except Exception as e:  # pragma: no cover - reported, never fatal for the main line
+        res["formats_28672x8192"] = {"error": f"{type(e).__name__}: {e}"[:200]}
     return res
 
 

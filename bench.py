@@ -487,6 +487,38 @@ def run_other_workloads(peaks, dev):
         del Wd, fc, fs, fS, q8, c1, mu
     except Exception as e:  # pragma: no cover - reported, never fatal for the main line
         res["formats_28672x8192"] = {"error": f"{type(e).__name__}: {e}"[:200]}
+    del d, codes, absmax, A, B, c_out, a_out
+    torch.cuda.empty_cache()
+    # The gated-MLP block (x [8192, 8192], F = 28672, r = 64 per layer): gate+up as one stacked QLoRA layer,
+    # SwiGLU, down; forward, then backward from the saved activations.  Tens of milliseconds per pass, so its
+    # fraction is taken against the sustained bf16 peak.
+    try:
+        from qlora_fine_tuning_blockwise_b200.mlp import QLoRAGatedMLP
+        c = I.make_chain_inputs()
+        Ls = c["layers"]
+
+        def on(t):
+            return (t if isinstance(t, torch.Tensor) else torch.from_numpy(t)).to(dev).contiguous()
+        block = QLoRAGatedMLP(on(Ls["gate"]["W"]), on(Ls["up"]["W"]), on(Ls["down"]["W"]), on(Ls["gate"]["A"]),
+                              on(Ls["gate"]["B"]), on(Ls["up"]["A"]), on(Ls["up"]["B"]), on(Ls["down"]["A"]),
+                              on(Ls["down"]["B"]), c["s"])
+        x, dy = on(c["x"]), on(c["dy"])
+        del c, Ls
+        torch.cuda.empty_cache()
+        f_ms = timeit(lambda: block.forward(x), reps=5)
+        _, saved = block.forward(x)
+        b_ms = timeit(lambda: block.backward(dy, x, saved), reps=5)
+        ff, fb = QLoRAGatedMLP.flops(x.shape[0], block.D, block.F, block.r)
+        sus = peaks["bf16_tflops_sustained"] * 1e12
+        res[I.CHAIN["name"]] = {"fwd_ms": round(f_ms, 3), "fwd_tflops": round(ff / (f_ms * 1e-3) / 1e12, 1),
+                                "fwd_frac_of_sustained": round(ff / (f_ms * 1e-3) / sus, 4),
+                                "bwd_ms": round(b_ms, 3), "bwd_tflops": round(fb / (b_ms * 1e-3) / 1e12, 1),
+                                "bwd_frac_of_sustained": round(fb / (b_ms * 1e-3) / sus, 4),
+                                "step_tflops": round((ff + fb) / ((f_ms + b_ms) * 1e-3) / 1e12, 1)}
+        del block, x, dy, saved
+        torch.cuda.empty_cache()
+    except Exception as e:  # pragma: no cover - reported, never fatal for the main line
+        res[I.CHAIN["name"]] = {"error": f"{type(e).__name__}: {e}"[:200]}
     return res
 
 

@@ -129,3 +129,25 @@ def test_merge_rejects_bad_arguments_on_host(L):
     assert lib.qlora_merge_lora_nf4(4, 64, 8, p, p, p, p, 2.0, None, p, None) == L.QL_ERR_INVALID_ARG
     assert lib.qlora_merge_lora(4, 64, 8, ctypes.c_void_p(FAKE + 2), p, p, p, 2.0, 0, p, None) == \
         L.QL_ERR_INVALID_ARG  # misaligned codes
+
+
+def test_format_conversions_reject_bad_arguments_on_host(L):
+    lib = L.lib()
+    p = ctypes.c_void_p(FAKE)
+    bad = ctypes.c_void_p(FAKE + 4)
+    # double quantization: empty, null, misaligned, too little scratch
+    need = lib.nf4_double_quantize_scratch_bytes(1000)
+    assert need == 4 * 8 and lib.nf4_double_quantize_scratch_bytes(0) == 0
+    assert lib.nf4_double_quantize(p, 0, p, p, p, p, need, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nf4_double_quantize(None, 1000, p, p, p, p, need, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nf4_double_quantize(p, 1000, p, p, bad, p, need, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nf4_double_quantize(p, 1000, p, p, p, p, need - 1, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nf4_double_dequantize(p, p, None, 1000, p, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nf4_double_dequantize(p, p, p, -5, p, None) == L.QL_ERR_INVALID_ARG
+    # NVFP4: numel not a multiple of 16, null, misaligned, bad dtype
+    assert lib.nvfp4_quantize(p, 24, p, p, p, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nvfp4_quantize(p, 32, p, None, p, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nvfp4_quantize(bad, 32, p, p, p, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nvfp4_dequantize(p, p, p, 32, 9, p, None) == L.QL_ERR_INVALID_ARG
+    assert lib.nvfp4_dequantize(p, p, p, 0, 0, p, None) == L.QL_ERR_INVALID_ARG
+    assert L.formats_launch_count() == 0  # nothing above reached a launch

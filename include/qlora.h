@@ -43,7 +43,7 @@ extern "C" {
 typedef enum {
   QL_OK = 0,
   QL_ERR_INVALID_ARG = 1,  /* bad shape, null or misaligned pointer, too-small workspace */
-  QL_ERR_UNSUPPORTED = 2,  /* valid parameters this build does not implement (e.g. blocksize != 64) */
+  QL_ERR_UNSUPPORTED = 2,  /* valid parameters the library does not implement (e.g. blocksize != 64) */
   QL_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
   QL_ERR_TIMEOUT = 4       /* a kernel's bounded wait expired (reported by ql_get_device_error) */
 } ql_status;

@@ -7,13 +7,18 @@ groups <= A ring).  This test models the protocol -- barrier phases and parity w
 defines them, every warp role (the four warps of a dequantizer group run independently), and the asynchronous
 landing of copies and completion of MMAs at random times -- and runs it under random schedules:
 
-  * with the depths the kernel uses, every consumer must read the stage it expects, the MMAs' operands must stay
-    intact until their completion is signalled, and the schedule must never deadlock;
-  * with a planted violation (more dequantizer groups than A slots, as in an earlier build that hung its waits
+  * with the depths the kernel uses -- read from the kernel's own configuration for every dequantizing
+    instantiation (tests/ring_depths.cu, built for the host) -- every consumer must read the stage it expects,
+    the MMAs' operands must stay intact until their completion is signalled, and the schedule must never
+    deadlock;
+  * with a planted violation (more dequantizer groups than A slots, a configuration that once hung its waits
     on the GPU) some schedule must break one of those properties.
 """
 
+import os
 import random
+import shutil
+import subprocess
 from dataclasses import dataclass, field
 
 import pytest
@@ -264,3 +269,29 @@ def test_relations_at_their_boundary_hold(QS, AS, G):
     for seed in range(100):
         errs = run(cfg, seed)
         assert not errs, (seed, errs[:3])
+
+
+def kernel_depths(tmpdir):
+    """(BN, AM, KB, QS, AS, BS, G, acc_bufs) of every dequantizing instantiation, from the kernel's own
+    configuration (tests/ring_depths.cu, built for the host with nvcc)."""
+    nvcc = os.environ.get("NVCC") or shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    exe = os.path.join(tmpdir, "ring_depths")
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "ring_depths.cu")
+    subprocess.run([nvcc, "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "--expt-relaxed-constexpr",
+                    "-o", exe, src], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    return [tuple(int(v) for v in line.split()) for line in out.strip().splitlines()]
+
+
+def test_every_instantiation_is_safe_under_random_schedules(tmp_path):
+    """The model with the depths each dequantizing kernel instantiation actually uses (not a copy of them)."""
+    rows = kernel_depths(str(tmp_path))
+    assert len(rows) == 13
+    for BN, AM, KB, QS, AS, BS, G, acc in sorted({r for r in rows}):
+        assert QS >= AS + G and G <= AS, (BN, AM, KB)
+        cfg = Cfg(QS, AS, BS, G, UNITS, acc_bufs=acc)
+        for seed in range(12):
+            errs = run(cfg, 1000 + seed)
+            assert not errs, ((BN, AM, KB), seed, errs[:3])

@@ -32,6 +32,8 @@ R23 packing: element 2j of the flat row-major weight sits in the LOW nibble of b
 Storage: 0.5 byte per weight for the codes plus 1 byte per 16 weights for the scales (0.5625 byte per weight,
 the same as NF4 with fp32 absmax per 64) plus one fp32 per tensor.
 
+R24 (the FP4 tensor-core form of the layer, ``fp4_linear_forward``): see the section at the end.
+
 Pins: ``tests/test_oracle_nvfp4.py``.
 """
 
@@ -164,3 +166,32 @@ def nvfp4_dequantize(codes: np.ndarray, scales: np.ndarray, S, numel: int, block
     v = e2m1_table()[nvfp4_unpack(codes)[:numel]]
     D = np.repeat(nvfp4_block_scales(scales, S), block)[:numel]
     return _f32(v * D.astype(np.float64))
+
+
+# --------------------------------------------------------------------------------------------------
+# The FP4 tensor-core form of the layer (R24)
+# --------------------------------------------------------------------------------------------------
+#
+# R24 the block-scaled FP4 MMA multiplies two E2M1 operands, so in that form the activations entering the base
+#     product are NVFP4-quantized too, by the same rule as the weight (R20-R22, blocks of 16 along K, their own
+#     tensor scale).  The LoRA branch keeps the unquantized activations (the adapters are trained in bf16).
+#         y = q(x) q(W)^T + s (x A^T) B^T,   q = NVFP4 quantize-then-dequantize,
+#     in fp64 from the dequantized fp32 operands.
+
+
+def nvfp4_roundtrip(a: np.ndarray) -> np.ndarray:
+    """q(a): the fp32 values a [rows, K] takes after NVFP4 quantization and dequantization (K % 16 == 0)."""
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    codes, scales, S = nvfp4_quantize(a.reshape(-1))
+    return nvfp4_dequantize(codes, scales, S, a.size).reshape(a.shape)
+
+
+def fp4_linear_forward(x, W, A, B, s: float) -> np.ndarray:
+    """y [M, N] in fp64 for the FP4 tensor-core form (R24): x [M, K] (bf16 values), W [N, K] fp32."""
+    xq = nvfp4_roundtrip(x).astype(np.float64)
+    wq = nvfp4_roundtrip(W).astype(np.float64)
+    x64 = np.asarray(x, dtype=np.float64)
+    y = xq @ wq.T
+    if A is not None and np.asarray(A).shape[0] > 0:
+        y = y + float(s) * ((x64 @ np.asarray(A, dtype=np.float64).T) @ np.asarray(B, dtype=np.float64).T)
+    return y

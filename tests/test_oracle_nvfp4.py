@@ -195,3 +195,56 @@ def test_planted_mistakes_are_caught(mistake):
         n = np.array([2.5, 5.0, 0.25], np.float32)
         away = np.array([3.0, 6.0, 0.5])  # ties away from zero
         assert not np.array_equal(F.e2m1_table()[F.e2m1_code_of(n)], away)
+
+
+# ------------------------------------------------------------------ the FP4 tensor-core form (R24)
+
+
+def grid_tensor(rows, cols, seed):
+    """A tensor on the NVFP4 grid (as in test_worked_tensor_round_trips_exactly): each block holds a +-6 and has a
+    normal E4M3 scale, one block reaches 448, so S = 2^-10 and q is the identity."""
+    rng = np.random.default_rng(seed)
+    nblk = rows * cols // 16
+    sb = rng.integers(0x08, 0x7E, nblk).astype(np.uint8)
+    sb[0] = 0x7E
+    codes = rng.integers(0, 16, (nblk, 16)).astype(np.uint8)
+    codes[:, 5] = 0x7
+    codes[codes == 0x8] = 0x0
+    sval = np.array([D.e4m3_value(int(c)) for c in sb])
+    return (F.e2m1_table()[codes] * (sval * 2.0 ** -10)[:, None]).astype(np.float32).reshape(rows, cols)
+
+
+def test_fp4_forward_on_grid_operands_is_the_plain_product():
+    x, W = grid_tensor(4, 64, 1), grid_tensor(6, 64, 2)
+    assert np.array_equal(F.nvfp4_roundtrip(x), x) and np.array_equal(F.nvfp4_roundtrip(W), W)
+    y = F.fp4_linear_forward(x, W, None, None, 2.0)
+    assert np.array_equal(y, x.astype(np.float64) @ W.astype(np.float64).T)
+
+
+def test_fp4_forward_lora_branch_uses_unquantized_activations():
+    """B = 0 leaves the quantized base product; the LoRA term is s (x A^T) B^T with the original x."""
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((5, 64))).astype(np.float32)
+    W = (rng.standard_normal((7, 64)) * 0.02).astype(np.float32)
+    A = rng.standard_normal((2, 64)).astype(np.float32)
+    B = rng.standard_normal((7, 2)).astype(np.float32)
+    base = F.fp4_linear_forward(x, W, None, None, 2.0)
+    assert np.array_equal(F.fp4_linear_forward(x, W, A, np.zeros_like(B), 2.0), base)
+    lora = F.fp4_linear_forward(x, W, A, B, 2.0) - base
+    ref = 2.0 * (x.astype(np.float64) @ A.T.astype(np.float64)) @ B.T.astype(np.float64)
+    assert np.allclose(lora, ref, rtol=1e-12, atol=1e-12)
+    # and it is not the quantized activations' product
+    xq = F.nvfp4_roundtrip(x).astype(np.float64)
+    assert not np.allclose(lora, 2.0 * (xq @ A.T.astype(np.float64)) @ B.T.astype(np.float64), rtol=1e-6)
+
+
+def test_fp4_forward_error_against_the_unquantized_product():
+    """On normal operands the FP4 form stays within the sum of the two operands' quantization errors: its
+    relative Frobenius distance from x W^T is of the order of sqrt(2) times NVFP4's relative rms error."""
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((64, 512)).astype(np.float32)
+    W = (rng.standard_normal((96, 512)) * 0.015).astype(np.float32)
+    y = F.fp4_linear_forward(x, W, None, None, 1.0)
+    ref = x.astype(np.float64) @ W.astype(np.float64).T
+    rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert 0.05 < rel < 0.2

@@ -1,0 +1,36 @@
+"""The reference arm of bench.py on the CPU: one JSON line with the contract's keys, and silent non-zero ranks."""
+
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+        "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
+
+
+def run(env_extra=None):
+    env = dict(os.environ, **(env_extra or {}))
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                           "--warmup", "3", "--ref-tokens", "16"], capture_output=True, text=True, env=env,
+                          timeout=600, cwd=ROOT)
+
+
+def test_reference_arm_prints_one_contract_line():
+    p = run()
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert KEYS <= set(out)
+    assert out["impl"] == "reference" and out["value"] > 0 and out["higher_is_better"] is True
+    assert out["config"]["workload"] == "attn_2048x4096x4096_r16"
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] >= 1
+    assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["d2h_bytes_per_step"] == 0
+    assert out["e2e"]["value"] == out["value"]
+
+
+def test_reference_arm_other_ranks_exit_silently():
+    p = run({"RANK": "1", "WORLD_SIZE": "2"})
+    assert p.returncode == 0 and p.stdout.strip() == ""

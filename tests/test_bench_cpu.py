@@ -74,3 +74,22 @@ def test_committed_traffic_record():
     if rec["source_sha"] != b.kernel_source_sha():
         pytest.skip("traffic recorded before the latest kernel change: re-capture it on a B200")
     assert b.load_traffic() == rec["kernels"]
+
+
+def test_clock_summary_parses_samples_and_reasons():
+    """nvidia-smi csv lines (noheader, nounits) -> median SM clock, max clock and the active throttle reasons."""
+    b = load_bench()
+    c = b.ClockSampler(0)
+    c.lines = [
+        "0, 1800, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1500, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1700, 1965, 950.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+    ]
+    s = c.summary()
+    assert s["sm_mhz"] == 1700.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+    c.lines = ["0, 1200, 1965, 500, 0x8, Not Active, Active, Not Active, Not Active"]
+    assert c.summary()["reasons"] == ["hw_thermal_slowdown"]
+    c.lines = []
+    assert c.summary()["reasons"] == ["unsampled"]

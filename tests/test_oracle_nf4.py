@@ -84,6 +84,62 @@ def test_codebook_golden_fixture():
     assert np.array_equal(np.array(vals, dtype=np.float32).view(np.uint32), O.nf4_codebook().view(np.uint32))
 
 
+def _paper_table() -> np.ndarray:
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "nf4_qlora_paper.txt")
+    vals = []
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if line:
+            idx, dec = line.split()
+            assert int(idx) == len(vals)
+            vals.append(float(dec))
+    assert len(vals) == 16
+    return np.array(vals, dtype=np.float64)
+
+
+def _paper_mismatch(table: np.ndarray) -> float:
+    """Largest relative difference between a 16-level table and the printed NF4 values (absolute at 0)."""
+    ref = _paper_table()
+    t = np.asarray(table, dtype=np.float64)
+    return float(np.max(np.abs(t - ref) / np.maximum(np.abs(ref), 1.0e-30 + (ref == 0))))
+
+
+PAPER_RTOL = 1.0e-6  # the printed values are fp32 levels written out in decimal; the rule reproduces them
+
+
+def test_codebook_matches_the_published_nf4_values():
+    """The level set equals the 16 values printed in the QLoRA paper (Appendix E), the public definition of
+    NF4 that reading R1 follows -- a pin from outside the oracle, not a restatement of its formula."""
+    c = O.nf4_codebook()
+    assert _paper_mismatch(c) <= PAPER_RTOL
+    # within a few fp32 ulps of the printed values, level by level
+    ref32 = _paper_table().astype(np.float32)
+    assert np.max(np.abs(c.view(np.int32).astype(np.int64) - ref32.view(np.int32).astype(np.int64))) <= 8
+
+
+@pytest.mark.parametrize("mistake", ["delta_1_32", "delta_1_30", "nine_point_negative_grid", "eight_point_positive_grid",
+                                     "uniform_instead_of_normal_quantiles"])
+def test_codebook_pin_catches_planted_mistakes(monkeypatch, mistake):
+    """Each plausible slip in the construction moves some level by far more than the pin's tolerance."""
+    if mistake == "delta_1_32":
+        monkeypatch.setattr(O, "NF4_DELTA", 1.0 / 32.0)
+    elif mistake == "delta_1_30":
+        monkeypatch.setattr(O, "NF4_DELTA", 1.0 / 30.0)
+    elif mistake == "uniform_instead_of_normal_quantiles":
+        monkeypatch.setattr(O, "normal_quantile", lambda p: p - 0.5)
+    else:
+        top = 1.0 - O.NF4_DELTA
+
+        def probs():
+            npos, nneg = {"nine_point_negative_grid": (8, 8), "eight_point_positive_grid": (7, 7)}[mistake]
+            pos = [top + i * (0.5 - top) / npos for i in range(8)]
+            neg = [top + i * (0.5 - top) / nneg for i in range(7)]
+            return pos, neg
+        monkeypatch.setattr(O, "nf4_probabilities", probs)
+    assert _paper_mismatch(O.nf4_codebook()) > 100 * PAPER_RTOL
+
+
 # ---------------------------------------------------------------------------------------------- quantize
 
 

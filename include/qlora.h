@@ -43,7 +43,7 @@ extern "C" {
 typedef enum {
   QL_OK = 0,
   QL_ERR_INVALID_ARG = 1,  /* bad shape, null or misaligned pointer, too-small workspace */
-  QL_ERR_UNSUPPORTED = 2,  /* valid parameters the library does not implement (e.g. blocksize != 64) */
+  QL_ERR_UNSUPPORTED = 2,  /* valid parameters this build does not implement (e.g. blocksize != 64) */
   QL_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed */
   QL_ERR_TIMEOUT = 4       /* a kernel's bounded wait expired (reported by ql_get_device_error) */
 } ql_status;
@@ -158,8 +158,9 @@ QL_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, 
  *               pass it to qlora_linear_bwd to skip recomputing it.
  *   workspace, ws_bytes  device scratch of at least qlora_workspace_bytes(M,N,K,r,QL_PASS_FWD) bytes
  *               (may be NULL when that is 0).
- * Products run on the tensor cores in bf16 with fp32 accumulation; deq(W) is formed in shared memory
- * tile by tile and never written to global memory.  The result is deterministic for given sizes.
+ * Products run on the tensor cores in bf16 with fp32 accumulation; deq(W) is formed tile by tile in tensor
+ * memory (TMEM), where the MMA reads it, and never written to global memory.  The result is deterministic
+ * for given sizes.
  */
 QL_API ql_status qlora_linear_fwd(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x, const uint8_t* codes,
                            const float* absmax, const uint16_t* A, const uint16_t* B, float s, uint16_t* y,
@@ -174,10 +175,13 @@ QL_API ql_status qlora_linear_fwd(int64_t M, int64_t N, int64_t K, int64_t r, co
  *   compiled into the library, which every GPU that loads the library holds until the process exits.
  *   Sizes whose qlora_workspace_bytes(M,N,K,r,QL_PASS_FWD) exceeds 8 MiB (8388608 bytes) return
  *   QL_ERR_INVALID_ARG before any launch.  No cudaMalloc, cudaFree or allocating routine is called.
- *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that device
- *   current; make that first call before any stream capture.  All calls share the one array and it keeps
- *   the last call's contents (the forward overwrites every scratch byte it reads), so calls that overlap on
- *   the GPU -- on different streams, or from several threads -- race; serialize them.
+ *   Every call looks up the array's device address in the current context (cudaGetSymbolAddress, with the
+ *   device current), since the address belongs to the context: it changes after cudaDeviceReset, and a
+ *   non-primary context has its own copy.  The first call in a context also loads every kernel the forward
+ *   can launch (module loading may allocate), so make that first call before any stream capture.  All
+ *   calls share the one array and it keeps the last call's contents (the forward overwrites every scratch
+ *   byte it reads), so calls that overlap on the GPU -- on different streams, or from several threads --
+ *   race; serialize them.
  */
 QL_API ql_status qlora_linear_fwd_noalloc(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x,
                                           const uint8_t* codes, const float* absmax, const uint16_t* A,
@@ -232,6 +236,72 @@ QL_API ql_status qlora_swiglu_gated_fwd(int64_t M, int64_t F, const uint16_t* gu
  */
 QL_API ql_status qlora_swiglu_gated_bwd(int64_t M, int64_t F, const uint16_t* dh, const uint16_t* gu,
                                         uint16_t* dgu, void* stream);
+
+/* ------------------------------------------------------------------------------------------------------
+ * Layer calls on a weight in any supported format.
+ * ------------------------------------------------------------------------------------------------------ */
+
+typedef enum { QL_W_NF4 = 0, QL_W_NF4_DQ = 1, QL_W_NVFP4 = 2 } ql_wformat;
+
+/* A frozen base weight W [N,K] (K a multiple of 64); all pointers device pointers, 16-byte aligned.
+ *   QL_W_NF4     codes [N*K/2] (nf4_quantize), absmax [N*K/64] fp32.
+ *   QL_W_NF4_DQ  codes, and the double-quantized constants of nf4_double_quantize: code8 [N*K/64] (readable to
+ *                a multiple of 4 bytes), c1 [ceil(N*K/64/256)] fp32, mu [1] fp32.
+ *   QL_W_NVFP4   codes [N*K/2] and scales [N*K/16] of nvfp4_quantize, tensor_scale [1] fp32.
+ * Pointers a format does not use are ignored. */
+typedef struct {
+  int format; /* ql_wformat */
+  const uint8_t* codes;
+  const float* absmax;
+  const uint8_t* code8;
+  const float* c1;
+  const float* mu;
+  const uint8_t* scales;
+  const float* tensor_scale;
+} ql_weight;
+
+/* qlora_linear_fwd / qlora_linear_bwd on a ql_weight: the same operation, layouts, workspace and errors, with
+ * deq(W) the weight's own dequantization (NF4: level * absmax; NF4_DQ: level * absmax' with the constants'
+ * double dequantization; NVFP4: E2M1 value * decoded group scale).  QL_ERR_INVALID_ARG for an unknown format or
+ * a null or misaligned pointer the format uses. */
+QL_API ql_status qlora_linear_fwd_w(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x, const ql_weight* w,
+                                    const uint16_t* A, const uint16_t* B, float s, uint16_t* y, uint16_t* su_out,
+                                    void* workspace, size_t ws_bytes, void* stream);
+QL_API ql_status qlora_linear_bwd_w(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* dy, const uint16_t* x,
+                                    const ql_weight* w, const uint16_t* A, const uint16_t* B, float s,
+                                    const uint16_t* su_in, uint16_t* dx, float* dA, float* dB, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------------------
+ * Gated MLP with the SwiGLU fused into the projections' epilogues.
+ *
+ * The gate/up projection is one layer over the stacked weight [2F, K] in the INTERLEAVED row order: within
+ * every 32 rows, the 16 gate rows of features 16q .. 16q + 15, then the 16 up rows of the same features
+ * (gate feature f at row 32 (f / 16) + f % 16, up feature f 16 rows below).  Its output gu [M, 2F] has the
+ * same column order.  F % 16 == 0.
+ * ------------------------------------------------------------------------------------------------------ */
+
+/* Workspace of the gated calls (the forward: that of qlora_linear_fwd; the down backward: that of
+ * qlora_linear_bwd plus, when its dX GEMM splits its contraction, a dh buffer of M*F bf16). */
+QL_API size_t qlora_gated_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass);
+
+/* Forward of the interleaved gate/up layer (qlora_linear_fwd with N = 2F) that also writes
+ * h [M, F] bf16 = silu(g) * up, g and up the bf16 values written to gu.  Bit-identical to qlora_linear_fwd
+ * followed by the SwiGLU of gu. */
+QL_API ql_status qlora_gate_up_fwd_swiglu(int64_t M, int64_t F, int64_t K, int64_t r, const uint16_t* x,
+                                          const uint8_t* codes, const float* absmax, const uint16_t* A,
+                                          const uint16_t* B, float s, uint16_t* gu, uint16_t* h, uint16_t* su_out,
+                                          void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of the down projection (W [N, F], input h) whose input gradient dh goes straight into the SwiGLU
+ * backward: dgu [M, 2F] (interleaved) = (dh * up * silu'(g), dh * silu(g)) with dh rounded to bf16 and g, up
+ * read from gu.  dA, dB as in qlora_linear_bwd.  Bit-identical to qlora_linear_bwd (dX = dh) followed by the
+ * SwiGLU backward. */
+QL_API ql_status qlora_down_bwd_dswiglu(int64_t M, int64_t N, int64_t F, int64_t r, const uint16_t* dy,
+                                        const uint16_t* h, const uint8_t* codes, const float* absmax,
+                                        const uint16_t* A, const uint16_t* B, float s, const uint16_t* su,
+                                        const uint16_t* gu, uint16_t* dgu, float* dA, float* dB, void* workspace,
+                                        size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------------------
  * Weight-format conversions (their own translation unit; their own launch counter and device error word).

@@ -5,6 +5,7 @@
 
 #include "nf4_table.cuh"
 #include "ptx.cuh"
+#include "swiglu.cuh"
 
 namespace qlora {
 
@@ -165,7 +166,6 @@ __global__ void reduce_splits_kernel(const float* __restrict__ ws, long long sla
   }
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
 __global__ void swiglu_fwd_kernel(const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ u,
                                   __nv_bfloat16* __restrict__ h, long long numel) {
@@ -173,7 +173,7 @@ __global__ void swiglu_fwd_kernel(const __nv_bfloat16* __restrict__ g, const __n
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < numel; e += stride) {
     const float gv = __bfloat162float(g[e]);
     const float uv = __bfloat162float(u[e]);
-    h[e] = __float2bfloat16_rn(silu_f(gv) * uv);
+    h[e] = __float2bfloat16_rn(swiglu_h(gv, uv));
   }
 }
 
@@ -185,11 +185,10 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* dh, const __nv_bfloat16* 
     const float gv = __bfloat162float(g[e]);
     const float uv = __bfloat162float(u[e]);
     const float dv = __bfloat162float(dh[e]);
-    const float sg = 1.0f / (1.0f + expf(-gv));
-    const float silu = gv * sg;
-    const float dsilu = sg * (1.0f + gv * (1.0f - sg));
-    dg[e] = __float2bfloat16_rn(dv * uv * dsilu);
-    du[e] = __float2bfloat16_rn(dv * silu);
+    float dgv, duv;
+    swiglu_grads(dv, gv, uv, dgv, duv);
+    dg[e] = __float2bfloat16_rn(dgv);
+    du[e] = __float2bfloat16_rn(duv);
   }
 }
 
@@ -211,7 +210,7 @@ __global__ void swiglu_gated_fwd_kernel(const __nv_bfloat16* __restrict__ gu, __
     for (int i = 0; i < 4; ++i) {
       const float2 g = __bfloat1622float2(g2[i]);
       const float2 u = __bfloat1622float2(u2[i]);
-      o2[i] = __floats2bfloat162_rn(silu_f(g.x) * u.x, silu_f(g.y) * u.y);
+      o2[i] = __floats2bfloat162_rn(swiglu_h(g.x, u.x), swiglu_h(g.y, u.y));
     }
     *reinterpret_cast<uint4*>(h + m * F + f) = out;
   }
@@ -239,13 +238,69 @@ __global__ void swiglu_gated_bwd_kernel(const __nv_bfloat16* __restrict__ dh, co
       const float2 d = __bfloat1622float2(d2[i]);
       const float2 g = __bfloat1622float2(g2[i]);
       const float2 u = __bfloat1622float2(u2[i]);
-      const float sx = 1.0f / (1.0f + expf(-g.x)), sy = 1.0f / (1.0f + expf(-g.y));
-      og2[i] = __floats2bfloat162_rn(d.x * u.x * (sx * (1.0f + g.x * (1.0f - sx))),
-                                     d.y * u.y * (sy * (1.0f + g.y * (1.0f - sy))));
-      ou2[i] = __floats2bfloat162_rn(d.x * (g.x * sx), d.y * (g.y * sy));
+      float gx, ux, gy, uy;
+      swiglu_grads(d.x, g.x, u.x, gx, ux);
+      swiglu_grads(d.y, g.y, u.y, gy, uy);
+      og2[i] = __floats2bfloat162_rn(gx, gy);
+      ou2[i] = __floats2bfloat162_rn(ux, uy);
     }
     *reinterpret_cast<uint4*>(dgu + m * 2 * F + f) = og;
     *reinterpret_cast<uint4*>(dgu + m * 2 * F + F + f) = ou;
+  }
+}
+
+// The same two steps over the interleaved gate/up layout (gate_pos / up_pos), for the calls whose GEMM splits
+// its contraction (the fused epilogues need the whole sum in one place).  8 consecutive features per thread.
+__global__ void swiglu_interleaved_fwd_kernel(const __nv_bfloat16* __restrict__ gu, __nv_bfloat16* __restrict__ h,
+                                              long long M, long long F) {
+  const long long groups = M * (F / 8);
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < groups; e += stride) {
+    const long long m = e / (F / 8), f = (e % (F / 8)) * 8;
+    const uint4 gv = *reinterpret_cast<const uint4*>(gu + m * 2 * F + gate_pos(f));
+    const uint4 uv = *reinterpret_cast<const uint4*>(gu + m * 2 * F + up_pos(f));
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+    const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&uv);
+    uint4 out;
+    __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 g = __bfloat1622float2(g2[i]);
+      const float2 u = __bfloat1622float2(u2[i]);
+      o2[i] = __floats2bfloat162_rn(swiglu_h(g.x, u.x), swiglu_h(g.y, u.y));
+    }
+    *reinterpret_cast<uint4*>(h + m * F + f) = out;
+  }
+}
+
+__global__ void swiglu_interleaved_bwd_kernel(const __nv_bfloat16* __restrict__ dh, const __nv_bfloat16* __restrict__ gu,
+                                              __nv_bfloat16* __restrict__ dgu, long long M, long long F) {
+  const long long groups = M * (F / 8);
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < groups; e += stride) {
+    const long long m = e / (F / 8), f = (e % (F / 8)) * 8;
+    const uint4 dv = *reinterpret_cast<const uint4*>(dh + m * F + f);
+    const uint4 gv = *reinterpret_cast<const uint4*>(gu + m * 2 * F + gate_pos(f));
+    const uint4 uv = *reinterpret_cast<const uint4*>(gu + m * 2 * F + up_pos(f));
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+    const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&uv);
+    uint4 og, ou;
+    __nv_bfloat162* og2 = reinterpret_cast<__nv_bfloat162*>(&og);
+    __nv_bfloat162* ou2 = reinterpret_cast<__nv_bfloat162*>(&ou);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 d = __bfloat1622float2(d2[i]);
+      const float2 g = __bfloat1622float2(g2[i]);
+      const float2 u = __bfloat1622float2(u2[i]);
+      float gx, ux, gy, uy;
+      swiglu_grads(d.x, g.x, u.x, gx, ux);
+      swiglu_grads(d.y, g.y, u.y, gy, uy);
+      og2[i] = __floats2bfloat162_rn(gx, gy);
+      ou2[i] = __floats2bfloat162_rn(ux, uy);
+    }
+    *reinterpret_cast<uint4*>(dgu + m * 2 * F + gate_pos(f)) = og;
+    *reinterpret_cast<uint4*>(dgu + m * 2 * F + up_pos(f)) = ou;
   }
 }
 

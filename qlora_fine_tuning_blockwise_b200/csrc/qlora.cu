@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -35,6 +36,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct DeviceInfo {
   int sms = 148;
   unsigned int* err = nullptr;
+  cudaStream_t side = nullptr;  // second stream for work that runs beside a GEMM (nullptr: none)
 };
 
 std::atomic<uint64_t> g_launches{0};
@@ -48,25 +50,37 @@ void prof_record(int which, int edge, cudaStream_t stream) {
   if (ev) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), stream);
 }
 
-DeviceInfo g_dev[kMaxDevices];
-bool g_dev_ready[kMaxDevices] = {};
+int g_dev_sms[kMaxDevices] = {};
+cudaStream_t g_dev_side[kMaxDevices] = {};
 std::mutex g_dev_mu;
 
-// Per-device constants, created on first use on that device (the current one).
+// The current device's SM count (cached per device: a property of the hardware) and the device address of
+// the error word.  That address belongs to the current context -- it changes after cudaDeviceReset, and a
+// non-primary context has its own copy -- so it is looked up on every call; once the library's module is
+// loaded in the context, the lookup allocates nothing.
 bool device_info(DeviceInfo* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  std::lock_guard<std::mutex> lk(g_dev_mu);
-  if (!g_dev_ready[dev]) {
-    DeviceInfo d;
-    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess) return false;
-    d.err = static_cast<unsigned int*>(p);
-    g_dev[dev] = d;
-    g_dev_ready[dev] = true;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (g_dev_sms[dev] <= 0) {
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return false;
+      // the side stream takes the lowest priority: the GEMM it runs beside keeps its SMs
+      int lowest = 0, highest = 0;
+      if (cudaDeviceGetStreamPriorityRange(&lowest, &highest) != cudaSuccess ||
+          cudaStreamCreateWithPriority(&g_dev_side[dev], cudaStreamNonBlocking, lowest) != cudaSuccess) {
+        g_dev_side[dev] = nullptr;
+        cudaGetLastError();
+      }
+      g_dev_sms[dev] = sms;
+    }
+    out->sms = g_dev_sms[dev];
+    out->side = g_dev_side[dev];
   }
-  *out = g_dev[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess || p == nullptr) return false;
+  out->err = static_cast<unsigned int*>(p);
   return true;
 }
 
@@ -125,6 +139,42 @@ struct Operand {  // a bf16 row-major matrix used through TMA
   int64_t rows = 0, cols = 0;
 };
 
+// dX through the transposing tensor-memory dequantizer (QLORA_DX_TMEM=1; off by default until measured)
+bool dx_tmem_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("QLORA_DX_TMEM");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
+
+// Cluster split-K for the skinny rank-r GEMMs (QLORA_CLUSTER_SPLITK=1; off by default until measured)
+bool cluster_splitk_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("QLORA_CLUSTER_SPLITK");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
+
+// CTA pairs for the 256-token fused GEMMs (QLORA_PAIRS=1; off by default until measured)
+bool pairs_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("QLORA_PAIRS");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
+
+// Grouped unit order (QLORA_GROUPED=0 turns it off, for comparison)
+bool grouped_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("QLORA_GROUPED");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 struct GemmCall {
   int am = A_TMA_K;
   bool b_mn = false;
@@ -134,15 +184,16 @@ struct GemmCall {
   int64_t rows = 0, cols = 0, k_total = 0;
   int n_extra = 0;
   int kb = 1;             // NF4 blocks per pipeline stage (4 only for token-light A_DEQ_TMEM)
+  bool pair = false;      // 2-SM MMA by CTA pairs (256-row tiles, each CTA holding half of the B tile)
   int splits = 1;
   int prof = -1;          // profiling-event slot recorded around this launch (-1: none)
-  int ctas = 148;         // persistent CTAs: at most one per SM
+  int ctas = 0;           // persistent CTAs: at most one per SM (0: as many as the GPU has SMs)
   UmmaArgs args{};
 };
 
-template <int BN, int AM, bool BMN, int KB = 1>
+template <int BN, int AM, bool BMN, int KB = 1, bool PAIR = false, int WF = WF_NF4, int EPI = EPI_PLAIN>
 cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
-  using C = UmmaCfg<BN, AM, BMN, KB>;
+  using C = UmmaCfg<BN, AM, BMN, KB, PAIR, EPI>;
   CUtensorMap tmA, tmB, tmBx, tmC;
   std::memset(&tmA, 0, sizeof(tmA));
   std::memset(&tmBx, 0, sizeof(tmBx));
@@ -152,7 +203,7 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
   if (BMN) {
     if (!make_map(&tmB, g.b.ptr, g.b.rows, g.b.cols, 2, 64, 64, true)) return cudaErrorInvalidValue;
   } else {
-    if (!make_map(&tmB, g.b.ptr, g.b.rows, g.b.cols, 2, 64, BN, true)) return cudaErrorInvalidValue;
+    if (!make_map(&tmB, g.b.ptr, g.b.rows, g.b.cols, 2, 64, C::kBRows, true)) return cudaErrorInvalidValue;
   }
   // A (TMA modes or LoRA extra)
   if (g.a.ptr) {
@@ -163,13 +214,19 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
     }
   }
   if (g.bx.ptr) {
-    if (!make_map(&tmBx, g.bx.ptr, g.bx.rows, g.bx.cols, 2, 64, BN, true)) return cudaErrorInvalidValue;
+    if (!make_map(&tmBx, g.bx.ptr, g.bx.rows, g.bx.cols, 2, 64, C::kBRows, true)) return cudaErrorInvalidValue;
   }
   if (C::kAbsTma) {
     // 4-block stages: codes 128 rows x 128 bytes (swizzled), absmax 128 rows x 4 values into tmA
     const int64_t N = g.args.w_rows, K = g.args.w_cols;
     if (!make_map(&tmC, g.codes, N, K / 2, 1, 128, 128, true)) return cudaErrorInvalidValue;
-    if (!make_map(&tmA, g.args.absmax, N, K / 64, 4, 4, 128, false)) return cudaErrorInvalidValue;
+    // the stage's scale words (128 rows x 16 bytes) into tmA: the fp32 absmax values or the NVFP4 group scales;
+    // the double-quantized constants come by cp.async instead
+    if constexpr (WF == WF_NF4) {
+      if (!make_map(&tmA, g.args.scale_words, N, K / 64, 4, 4, 128, false)) return cudaErrorInvalidValue;
+    } else if constexpr (WF == WF_NVFP4) {
+      if (!make_map(&tmA, g.args.scale_words, N, K / 16, 1, 16, 128, false)) return cudaErrorInvalidValue;
+    }
   } else if (C::kDeq) {
     const int64_t N = g.args.w_rows, K = g.args.w_cols;
     if (AM == A_DEQ_TMEM) {
@@ -178,51 +235,148 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
       if (!make_map(&tmC, g.codes, N, K / 2, 1, 64, 64, false)) return cudaErrorInvalidValue;
     }
   }
-  auto kern = umma_gemm_kernel<BN, AM, BMN, KB>;
+  auto kern = umma_gemm_kernel<BN, AM, BMN, KB, PAIR, WF, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int64_t units = static_cast<int64_t>(g.args.splits) * g.args.tiles_i * g.args.tiles_j;
-  dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, g.ctas)));
-  if (g.prof >= 0) prof_record(g.prof, 0, stream);
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmBx, tmC, g.args);
+  if constexpr (PAIR) {
+    // clusters of two CTAs, each pair walking the units; no more pairs than can be resident at once (a GPC with
+    // an odd number of free SMs leaves one idle), so no unit waits for a pair to retire
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(g.ctas & ~1));
+    int resident = 0;
+    if (cudaOccupancyMaxActiveClusters(&resident, kern, &cfg) != cudaSuccess || resident <= 0) {
+      cudaGetLastError();
+      resident = g.ctas / 2;
+    }
+    const int64_t pairs = std::min<int64_t>(units, std::min(resident, g.ctas / 2));
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    if (g.prof >= 0) prof_record(g.prof, 0, stream);
+    e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmBx, tmC, g.args);
+    if (e != cudaSuccess) return e;
+  } else if (!C::kDeq && g.args.cred > 1) {
+    // cluster split-K: one CTA per unit, the S splits of a tile in one cluster; every unit must be resident at
+    // once (the clusters reduce at the end), else the caller falls back to partial slabs
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(g.args.cred);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(units));
+    int resident = 0;
+    if (cudaOccupancyMaxActiveClusters(&resident, kern, &cfg) != cudaSuccess || resident <= 0 ||
+        static_cast<int64_t>(resident) * g.args.cred < units) {
+      cudaGetLastError();
+      return cudaErrorCooperativeLaunchTooLarge;
+    }
+    if (g.prof >= 0) prof_record(g.prof, 0, stream);
+    e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmBx, tmC, g.args);
+    if (e != cudaSuccess) return e;
+  } else {
+    dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, g.ctas)));
+    if (g.prof >= 0) prof_record(g.prof, 0, stream);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmBx, tmC, g.args);
+  }
   count_launch();
   if (g.prof >= 0) prof_record(g.prof, 1, stream);
   return cudaGetLastError();
 }
 
-template <int AM, bool BMN>
+template <int AM, bool BMN, int WF = WF_NF4>
 cudaError_t launch_bn(const GemmCall& g, cudaStream_t stream) {
   if constexpr (BMN) {
     switch (g.bn) {
-      case 64: return launch_umma<64, AM, BMN>(g, stream);
-      case 128: return launch_umma<128, AM, BMN>(g, stream);
-      case 256: return launch_umma<256, AM, BMN>(g, stream);
+      case 64: return launch_umma<64, AM, BMN, 1, false, WF>(g, stream);
+      case 128: return launch_umma<128, AM, BMN, 1, false, WF>(g, stream);
+      case 256: return launch_umma<256, AM, BMN, 1, false, WF>(g, stream);
       default: return cudaErrorInvalidValue;
     }
   } else {
     switch (g.bn) {
-      case 16: return launch_umma<16, AM, BMN>(g, stream);
-      case 32: return launch_umma<32, AM, BMN>(g, stream);
-      case 64: return launch_umma<64, AM, BMN>(g, stream);
-      case 128: return launch_umma<128, AM, BMN>(g, stream);
-      case 256: return launch_umma<256, AM, BMN>(g, stream);
+      case 16: return launch_umma<16, AM, BMN, 1, false, WF>(g, stream);
+      case 32: return launch_umma<32, AM, BMN, 1, false, WF>(g, stream);
+      case 64: return launch_umma<64, AM, BMN, 1, false, WF>(g, stream);
+      case 128: return launch_umma<128, AM, BMN, 1, false, WF>(g, stream);
+      case 256: return launch_umma<256, AM, BMN, 1, false, WF>(g, stream);
       default: return cudaErrorInvalidValue;
     }
   }
 }
 
-cudaError_t launch_gemm(const GemmCall& g, cudaStream_t stream) {
+// The dequantizing GEMMs, by weight format.
+template <int WF>
+cudaError_t launch_deq(const GemmCall& g, cudaStream_t stream) {
+  if (g.pair) {
+    if (g.bn != 256 || g.b_mn || g.kb != 1) return cudaErrorInvalidValue;
+    if (g.am == A_DEQ_TMEM) return launch_umma<256, A_DEQ_TMEM, false, 1, true, WF>(g, stream);
+    if (g.am == A_DEQ_MN) return launch_umma<256, A_DEQ_MN, false, 1, true, WF>(g, stream);
+    if constexpr (WF == WF_NF4) {
+      if (g.am == A_DEQ_TMEM_T) return launch_umma<256, A_DEQ_TMEM_T, false, 1, true, WF>(g, stream);
+    }
+    return cudaErrorInvalidValue;
+  }
   if (g.am == A_DEQ_TMEM && !g.b_mn && g.kb == 4) {
     switch (g.bn) {
-      case 16: return launch_umma<16, A_DEQ_TMEM, false, 4>(g, stream);
-      case 32: return launch_umma<32, A_DEQ_TMEM, false, 4>(g, stream);
-      case 64: return launch_umma<64, A_DEQ_TMEM, false, 4>(g, stream);
+      case 16: return launch_umma<16, A_DEQ_TMEM, false, 4, false, WF>(g, stream);
+      case 32: return launch_umma<32, A_DEQ_TMEM, false, 4, false, WF>(g, stream);
+      case 64: return launch_umma<64, A_DEQ_TMEM, false, 4, false, WF>(g, stream);
       default: return cudaErrorInvalidValue;
     }
   }
   if (g.kb != 1) return cudaErrorInvalidValue;
-  if (g.am == A_DEQ_TMEM && !g.b_mn) return launch_bn<A_DEQ_TMEM, false>(g, stream);
-  if (g.am == A_DEQ_MN && !g.b_mn) return launch_bn<A_DEQ_MN, false>(g, stream);
+  if (g.am == A_DEQ_TMEM && !g.b_mn) return launch_bn<A_DEQ_TMEM, false, WF>(g, stream);
+  if (g.am == A_DEQ_MN && !g.b_mn) return launch_bn<A_DEQ_MN, false, WF>(g, stream);
+  if constexpr (WF == WF_NF4) {
+    if (g.am == A_DEQ_TMEM_T && !g.b_mn) return launch_bn<A_DEQ_TMEM_T, false, WF>(g, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// The fused gated-MLP epilogues (NF4 weights): the gate/up forward (TMEM A) and the down projection's dX (MN A).
+template <int AM, int EPI>
+cudaError_t launch_epi(const GemmCall& g, cudaStream_t stream) {
+  switch (g.bn) {
+    case 16: return launch_umma<16, AM, false, 1, false, WF_NF4, EPI>(g, stream);
+    case 32: return launch_umma<32, AM, false, 1, false, WF_NF4, EPI>(g, stream);
+    case 64: return launch_umma<64, AM, false, 1, false, WF_NF4, EPI>(g, stream);
+    case 128: return launch_umma<128, AM, false, 1, false, WF_NF4, EPI>(g, stream);
+    case 256: return launch_umma<256, AM, false, 1, false, WF_NF4, EPI>(g, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_gemm(const GemmCall& g, cudaStream_t stream) {
+  if (g.args.epi != EPI_PLAIN) {
+    if (g.args.splits != 1 || g.kb != 1 || g.b_mn || g.pair || g.args.wfmt != WF_NF4) return cudaErrorInvalidValue;
+    if (g.args.epi == EPI_SWIGLU_FWD && g.am == A_DEQ_TMEM) return launch_epi<A_DEQ_TMEM, EPI_SWIGLU_FWD>(g, stream);
+    if (g.args.epi == EPI_DSWIGLU && g.am == A_DEQ_MN) return launch_epi<A_DEQ_MN, EPI_DSWIGLU>(g, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (g.am == A_DEQ_TMEM || g.am == A_DEQ_MN || g.am == A_DEQ_TMEM_T) {
+    switch (g.args.wfmt) {
+      case WF_NF4: return launch_deq<WF_NF4>(g, stream);
+      case WF_NF4_DQ: return launch_deq<WF_NF4_DQ>(g, stream);
+      case WF_NVFP4: return launch_deq<WF_NVFP4>(g, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (g.kb != 1) return cudaErrorInvalidValue;
   if (g.am == A_TMA_K && !g.b_mn) return launch_bn<A_TMA_K, false>(g, stream);
   if (g.am == A_TMA_K && g.b_mn) return launch_bn<A_TMA_K, true>(g, stream);
   if (g.am == A_TMA_MN && g.b_mn) return launch_bn<A_TMA_MN, true>(g, stream);
@@ -326,14 +480,41 @@ cudaError_t launch_reduce(const float* ws, int64_t slab, int nsplit, int64_t cou
   return cudaGetLastError();
 }
 
+// CTAs that give a persistent GEMM of `units` work units (`per_unit` CTAs each) the makespan it has on the whole
+// GPU: it takes ceil(units * per_unit / sms) waves either way, and with ceil(units / waves) units in flight its
+// last wave is as full as the others.  The SMs this leaves free can run other work in the meantime.
+int wave_exact_ctas(int64_t units, int per_unit, int sms) {
+  const int64_t slots = std::max<int64_t>(1, sms / per_unit);
+  const int64_t waves = cdiv(units, slots);
+  return static_cast<int>(cdiv(units, waves) * per_unit);
+}
+
 // Run a GEMM whose output is dense [count] in the final layout: direct when unsplit, else fp32 partials in
 // `part` then one reduction.
+// Tile rows per group of the unit order (0: tile columns fastest).  A wave of C concurrent units covering g tile
+// rows and C / g tile columns fetches about g weight tiles and C / g activation tiles; with w and a the bytes of
+// one of each (both proportional to the contraction length), g w + (C / g) a is smallest at g = sqrt(C a / w).
+// Grids of one wave, and outputs one tile column wide, keep the plain order.
+int unit_group(const GemmCall& g) {
+  if (!grouped_enabled() || g.args.tiles_j <= 1) return 0;
+  const int64_t concurrent = g.pair ? g.ctas / 2 : g.ctas;
+  const int64_t units = static_cast<int64_t>(g.args.splits) * g.args.tiles_i * g.args.tiles_j;
+  if (units <= concurrent) return 0;
+  const bool deq = g.am == A_DEQ_TMEM || g.am == A_DEQ_MN || g.am == A_DEQ_TMEM_T;
+  const double w_row_bytes = deq ? 0.5625 : 2.0;  // one weight row element: 4-bit code + its share of the scale
+  const double ratio = (g.bn * 2.0) / ((g.pair ? 256.0 : 128.0) * w_row_bytes);
+  int gi = static_cast<int>(std::lround(std::sqrt(static_cast<double>(concurrent) * ratio)));
+  if (gi < 1) gi = 1;
+  if (gi > g.args.tiles_i) gi = g.args.tiles_i;
+  return gi;
+}
+
 cudaError_t run_gemm(GemmCall g, void* out, bool out_bf16, float alpha, int64_t ls, int64_t cs, int64_t rows_lim,
                      int64_t cols_lim, int64_t count, float* part, unsigned int* err, cudaStream_t stream) {
-  g.ctas = plan_sms();
+  if (g.ctas <= 0) g.ctas = plan_sms();
   g.args.rows = static_cast<int>(g.rows);
   g.args.cols = static_cast<int>(g.cols);
-  g.args.tiles_i = static_cast<int>(cdiv(g.rows, 128));
+  g.args.tiles_i = static_cast<int>(cdiv(g.rows, g.pair ? 256 : 128));
   g.args.tiles_j = static_cast<int>(cdiv(g.cols, g.bn));
   g.args.k_stages = static_cast<int>(cdiv(g.k_total, 64 * g.kb));
   g.args.stages_per_split = static_cast<int>(cdiv(g.args.k_stages, g.splits));
@@ -345,12 +526,26 @@ cudaError_t run_gemm(GemmCall g, void* out, bool out_bf16, float alpha, int64_t 
   g.args.rows_lim = static_cast<int>(rows_lim);
   g.args.cols_lim = static_cast<int>(cols_lim);
   g.args.err = err;
+  g.args.group_i = unit_group(g);
   if (g.splits == 1) {
     g.args.out = out;
     g.args.out_bf16 = out_bf16 ? 1 : 0;
     g.args.alpha = alpha;
     g.args.split_stride = 0;
     return launch_gemm(g, stream);
+  }
+  const bool tma_mode = g.am == A_TMA_K || g.am == A_TMA_MN;
+  if (tma_mode && g.splits <= 8 && 128 % g.splits == 0 && cluster_splitk_enabled() &&
+      static_cast<int64_t>(g.splits) * g.args.tiles_i * g.args.tiles_j <= g.ctas) {
+    // the splits of a tile reduce inside their cluster: no slabs, no second launch
+    GemmCall c = g;
+    c.args.cred = g.splits;
+    c.args.out = out;
+    c.args.out_bf16 = out_bf16 ? 1 : 0;
+    c.args.alpha = alpha;
+    c.args.split_stride = 0;
+    const cudaError_t e = launch_gemm(c, stream);
+    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
   }
   g.args.out = part;
   g.args.out_bf16 = 0;
@@ -383,6 +578,268 @@ ql_status check_linear(int64_t M, int64_t N, int64_t K, int64_t r) {
   if (M < 0 || N < 1 || K < 64 || K % 64 != 0 || N % 8 != 0 || r < 0 || r > 256 || r % 8 != 0)
     return QL_ERR_INVALID_ARG;
   if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1) return QL_ERR_INVALID_ARG;
+  return QL_OK;
+}
+
+// The kernel's view of a weight descriptor: its format and the pointers that format uses.
+void set_weight(UmmaArgs& a, const ql_weight& w) {
+  a.wfmt = w.format == QL_W_NF4_DQ ? WF_NF4_DQ : w.format == QL_W_NVFP4 ? WF_NVFP4 : WF_NF4;
+  a.scale_words = w.format == QL_W_NF4_DQ ? static_cast<const void*>(w.code8)
+                  : w.format == QL_W_NVFP4 ? static_cast<const void*>(w.scales)
+                                           : static_cast<const void*>(w.absmax);
+  a.dq_c1 = w.c1;
+  a.dq_mu = w.mu;
+  a.fp4_S = w.tensor_scale;
+}
+
+ql_status check_weight(const ql_weight* w) {
+  if (!w || !w->codes || !aligned16(w->codes)) return QL_ERR_INVALID_ARG;
+  switch (w->format) {
+    case QL_W_NF4:
+      return w->absmax && aligned16(w->absmax) ? QL_OK : QL_ERR_INVALID_ARG;
+    case QL_W_NF4_DQ:
+      return w->code8 && w->c1 && w->mu && aligned16(w->code8) && aligned16(w->c1) && aligned16(w->mu)
+                 ? QL_OK
+                 : QL_ERR_INVALID_ARG;
+    case QL_W_NVFP4:
+      return w->scales && w->tensor_scale && aligned16(w->scales) && aligned16(w->tensor_scale) ? QL_OK
+                                                                                               : QL_ERR_INVALID_ARG;
+    default:
+      return QL_ERR_INVALID_ARG;
+  }
+}
+
+ql_weight nf4_weight(const uint8_t* codes, const float* absmax) {
+  ql_weight w = {};
+  w.format = QL_W_NF4;
+  w.codes = codes;
+  w.absmax = absmax;
+  return w;
+}
+
+// A fused epilogue for the main GEMM of a layer call (Epi in umma_gemm.cuh).
+struct EpiArgs {
+  int mode = EPI_PLAIN;
+  void* out2 = nullptr;
+  int64_t ls2 = 0, cs2 = 0;
+  const uint16_t* aux = nullptr;
+  int64_t aux_ld = 0;
+};
+
+ql_status linear_fwd_impl(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x, const ql_weight* w,
+                          const uint16_t* A, const uint16_t* B, float s, uint16_t* y, uint16_t* su_out,
+                          void* workspace, size_t ws_bytes, void* stream, const EpiArgs* epi) {
+  ql_status st = check_linear(M, N, K, r);
+  if (st != QL_OK) return st;
+  if (check_weight(w) != QL_OK) return QL_ERR_INVALID_ARG;
+  const ql_weight& wt = *w;
+  if (M == 0) return QL_OK;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return QL_ERR_INVALID_ARG;
+  if (r > 0 && (!A || !B || !aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
+  if (su_out && !aligned16(su_out)) return QL_ERR_INVALID_ARG;
+  const LinearPlan p = plan_linear(M, N, K, r, QL_PASS_FWD);
+  if (ws_bytes < p.total || (p.total > 0 && (!workspace || !aligned16(workspace)))) return QL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (!device_info(&d)) return QL_ERR_CUDA;
+  cudaStream_t cs = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* part = ws ? reinterpret_cast<float*>(ws + p.off_part) : nullptr;
+
+  uint16_t* su = su_out;
+  if (r > 0) {
+    if (!su) su = reinterpret_cast<uint16_t*>(ws + p.off_su);
+    cudaError_t e = run_su(M, K, r, x, A, s, su, p.s_su, part, d.err, cs);
+    if (e != cudaSuccess) return QL_ERR_CUDA;
+  }
+  GemmCall g;
+  g.am = A_DEQ_TMEM;
+  g.b_mn = false;
+  g.bn = p.bn_main;
+  g.b = {x, M, K};
+  if (r > 0) {
+    // the LoRA columns: A extra = rows of B (copied into tensor memory by the kernel), B extra = s x A^T
+    g.args.lora = B;
+    g.args.lora_ld = static_cast<int>(r);
+    g.args.lora_r = static_cast<int>(r);
+    g.bx = {su, M, r};
+  }
+  g.kb = fwd_stage_blocks(M, K);
+  g.pair = g.bn == 256 && g.kb == 1 && !epi && pairs_enabled();
+  if (r > 0) g.n_extra = static_cast<int>(cdiv(r, 64 * g.kb));
+  g.codes = wt.codes;
+  set_weight(g.args, wt);
+  g.args.w_rows = static_cast<int>(N);
+  g.args.w_cols = static_cast<int>(K);
+  g.args.w_kb = static_cast<int>(K / 64);
+  g.rows = N;
+  g.cols = M;
+  g.k_total = K;
+  g.splits = p.s_main;
+  g.prof = 0;
+  if (epi) {
+    g.args.epi = epi->mode;
+    g.args.out2 = epi->out2;
+    g.args.ls2 = epi->ls2;
+    g.args.cs2 = epi->cs2;
+  }
+  // D[i = n, j = m] -> y[m, n]
+  return status_of(run_gemm(g, y, true, 1.0f, 1, N, N, M, M * N, part, d.err, cs));
+}
+
+ql_status linear_bwd_impl(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* dy, const uint16_t* x,
+                          const ql_weight* w, const uint16_t* A, const uint16_t* B, float s, const uint16_t* su_in,
+                          uint16_t* dx, float* dA, float* dB, void* workspace, size_t ws_bytes, void* stream,
+                          const EpiArgs* epi) {
+  ql_status st = check_linear(M, N, K, r);
+  if (st != QL_OK) return st;
+  if (check_weight(w) != QL_OK) return QL_ERR_INVALID_ARG;
+  const ql_weight& wt = *w;
+  const bool want_da = r > 0 && dA, want_db = r > 0 && dB;
+  if ((dx && !aligned16(dx)) || (want_da && !aligned16(dA)) || (want_db && !aligned16(dB))) return QL_ERR_INVALID_ARG;
+  if (r > 0 && (!A || !B || !aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
+  if (su_in && !aligned16(su_in)) return QL_ERR_INVALID_ARG;
+  cudaStream_t cs = as_stream(stream);
+  if (M == 0) {
+    if (want_da && cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 4, cs) != cudaSuccess) return QL_ERR_CUDA;
+    if (want_db && cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 4, cs) != cudaSuccess) return QL_ERR_CUDA;
+    return QL_OK;
+  }
+  if (!dy || !aligned16(dy)) return QL_ERR_INVALID_ARG;
+  if ((want_da || want_db || (r > 0 && !su_in)) && (!x || !aligned16(x))) return QL_ERR_INVALID_ARG;
+  const LinearPlan p = plan_linear(M, N, K, r, QL_PASS_BWD);
+  if (ws_bytes < p.total || (p.total > 0 && (!workspace || !aligned16(workspace)))) return QL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (!device_info(&d)) return QL_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* part = ws ? reinterpret_cast<float*>(ws + p.off_part) : nullptr;
+  const int rp = rank_pad(r);
+
+  uint16_t* v = nullptr;
+  const uint16_t* su = su_in;
+  if (r > 0) {
+    // su = bf16(s x A^T), recomputed when the forward's copy is not supplied (needed by dB)
+    if (!su && want_db) {
+      uint16_t* su_ws = reinterpret_cast<uint16_t*>(ws + p.off_su);
+      if (run_su(M, K, r, x, A, s, su_ws, p.s_su, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
+      su = su_ws;
+    }
+    // v = bf16(s dY B) [M, r]: D[i = m, j] = sum_n dY[m, n] B[n, j]
+    v = reinterpret_cast<uint16_t*>(ws + p.off_v);
+    GemmCall g;
+    g.am = A_TMA_K;
+    g.b_mn = true;
+    g.bn = rp;
+    g.a = {dy, M, N};
+    g.b = {B, N, r};
+    g.rows = M;
+    g.cols = rp;
+    g.k_total = N;
+    g.splits = p.s_v;
+    if (run_gemm(g, v, true, s, r, 1, M, r, M * r, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
+  }
+  // dA and dB do not depend on dX: when the dX GEMM (unsplit) would leave its last wave partly empty, it runs
+  // on the fewest CTAs that keep its makespan, and dA, dB run beside it on the SMs it leaves free, on the
+  // device's side stream (forked from and joined back into the caller's stream).
+  const bool dx_pair = p.bn_main == 256 && !epi && pairs_enabled();
+  int dx_ctas = 0, side_sms = 0;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  if (dx && (want_da || want_db) && p.s_main == 1 && d.side) {
+    const int64_t units = cdiv(K, dx_pair ? 256 : 128) * cdiv(M, p.bn_main);
+    dx_ctas = wave_exact_ctas(units, dx_pair ? 2 : 1, d.sms);
+    side_sms = d.sms - dx_ctas;
+    if (side_sms >= 8 && cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventRecord(ev_fork, cs) == cudaSuccess && cudaStreamWaitEvent(d.side, ev_fork, 0) == cudaSuccess) {
+      // forked
+    } else {
+      if (ev_fork) cudaEventDestroy(ev_fork);
+      if (ev_join) cudaEventDestroy(ev_join);
+      ev_fork = ev_join = nullptr;
+      dx_ctas = side_sms = 0;
+      cudaGetLastError();
+    }
+  }
+  // on an error after the fork: release the events (they go once their work has run) and report
+  auto unfork = [&]() {
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    if (ev_join) cudaEventDestroy(ev_join);
+    return QL_ERR_CUDA;
+  };
+  const bool beside = side_sms > 0;
+  cudaStream_t gs = beside ? d.side : cs;  // the stream of dA and dB
+  if (dx) {
+    // dX^T: D[i = k, j = m] = sum_n deq(W)[n, k] dY[m, n]  (+ sum_j A[j, k] v[m, j])
+    GemmCall g;
+    // the transposing TMEM dequantizer when enabled (NF4 weights, plain epilogue, single CTAs)
+    g.am = dx_tmem_enabled() && !epi && wt.format == QL_W_NF4 ? A_DEQ_TMEM_T : A_DEQ_MN;
+    g.b_mn = false;
+    g.bn = p.bn_main;
+    g.pair = dx_pair;
+    g.ctas = dx_ctas;
+    g.b = {dy, M, N};
+    if (r > 0) {
+      // the LoRA rows: A extra = A [r, K] (copied into the MN-major tiles by the kernel), B extra = v
+      g.args.lora = A;
+      g.args.lora_ld = static_cast<int>(K);
+      g.args.lora_r = static_cast<int>(r);
+      g.bx = {v, M, r};
+      g.n_extra = static_cast<int>(cdiv(r, 64));
+    }
+    g.codes = wt.codes;
+    set_weight(g.args, wt);
+    g.args.w_rows = static_cast<int>(N);
+    g.args.w_cols = static_cast<int>(K);
+    g.args.w_kb = static_cast<int>(K / 64);
+    g.rows = K;
+    g.cols = M;
+    g.k_total = N;
+    g.splits = p.s_main;
+    g.prof = 1;
+    if (epi) {
+      g.args.epi = epi->mode;
+      g.args.out2 = epi->out2;
+      g.args.aux = epi->aux;
+      g.args.aux_ld = epi->aux_ld;
+    }
+    if (run_gemm(g, dx, true, 1.0f, 1, K, K, M, M * K, part, d.err, cs) != cudaSuccess) return unfork();
+  }
+  if (want_da) {
+    // dA^T: D[i = k, j] = sum_m x[m, k] v[m, j]  -> dA[j, k]
+    GemmCall g;
+    g.am = A_TMA_MN;
+    g.b_mn = true;
+    g.bn = rp;
+    g.a = {x, M, K};
+    g.b = {v, M, r};
+    g.rows = K;
+    g.cols = rp;
+    g.k_total = M;
+    g.splits = beside ? plan_splits(cdiv(K, 128), cdiv(M, 64), side_sms) : p.s_da;
+    g.ctas = side_sms;
+    if (run_gemm(g, dA, false, 1.0f, 1, K, K, r, r * K, part, d.err, gs) != cudaSuccess) return unfork();
+  }
+  if (want_db) {
+    // dB: D[i = n, j] = sum_m dY[m, n] su[m, j]
+    GemmCall g;
+    g.am = A_TMA_MN;
+    g.b_mn = true;
+    g.bn = rp;
+    g.a = {dy, M, N};
+    g.b = {su, M, r};
+    g.rows = N;
+    g.cols = rp;
+    g.k_total = M;
+    g.splits = beside ? plan_splits(cdiv(N, 128), cdiv(M, 64), side_sms) : p.s_db;
+    g.ctas = side_sms;
+    if (run_gemm(g, dB, false, 1.0f, r, 1, N, r, N * r, part, d.err, gs) != cudaSuccess) return unfork();
+  }
+  if (beside) {
+    // join: the caller's stream continues once dA and dB are done; the events go once they have fired
+    const bool ok = cudaEventRecord(ev_join, gs) == cudaSuccess && cudaStreamWaitEvent(cs, ev_join, 0) == cudaSuccess;
+    cudaEventDestroy(ev_fork);
+    cudaEventDestroy(ev_join);
+    if (!ok) return QL_ERR_CUDA;
+  }
   return QL_OK;
 }
 
@@ -503,164 +960,109 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass
   return plan_linear(M, N, K, r, pass).total;
 }
 
+
+
 ql_status qlora_linear_fwd(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x, const uint8_t* codes,
                            const float* absmax, const uint16_t* A, const uint16_t* B, float s, uint16_t* y,
                            uint16_t* su_out, void* workspace, size_t ws_bytes, void* stream) {
-  ql_status st = check_linear(M, N, K, r);
-  if (st != QL_OK) return st;
-  if (M == 0) return QL_OK;
-  if (!x || !codes || !absmax || !y || !aligned16(x) || !aligned16(codes) || !aligned16(absmax) || !aligned16(y))
-    return QL_ERR_INVALID_ARG;
-  if (r > 0 && (!A || !B || !aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
-  if (su_out && !aligned16(su_out)) return QL_ERR_INVALID_ARG;
-  const LinearPlan p = plan_linear(M, N, K, r, QL_PASS_FWD);
-  if (ws_bytes < p.total || (p.total > 0 && (!workspace || !aligned16(workspace)))) return QL_ERR_INVALID_ARG;
-  DeviceInfo d;
-  if (!device_info(&d)) return QL_ERR_CUDA;
-  cudaStream_t cs = as_stream(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* part = ws ? reinterpret_cast<float*>(ws + p.off_part) : nullptr;
+  const ql_weight w = nf4_weight(codes, absmax);
+  return linear_fwd_impl(M, N, K, r, x, &w, A, B, s, y, su_out, workspace, ws_bytes, stream, nullptr);
+}
 
-  uint16_t* su = su_out;
-  if (r > 0) {
-    if (!su) su = reinterpret_cast<uint16_t*>(ws + p.off_su);
-    cudaError_t e = run_su(M, K, r, x, A, s, su, p.s_su, part, d.err, cs);
-    if (e != cudaSuccess) return QL_ERR_CUDA;
-  }
-  GemmCall g;
-  g.am = A_DEQ_TMEM;
-  g.b_mn = false;
-  g.bn = p.bn_main;
-  g.b = {x, M, K};
-  if (r > 0) {
-    // the LoRA columns: A extra = rows of B (copied into tensor memory by the kernel), B extra = s x A^T
-    g.args.lora = B;
-    g.args.lora_ld = static_cast<int>(r);
-    g.args.lora_r = static_cast<int>(r);
-    g.bx = {su, M, r};
-  }
-  g.kb = fwd_stage_blocks(M, K);
-  if (r > 0) g.n_extra = static_cast<int>(cdiv(r, 64 * g.kb));
-  g.codes = codes;
-  g.args.absmax = absmax;
-  g.args.w_rows = static_cast<int>(N);
-  g.args.w_cols = static_cast<int>(K);
-  g.args.w_kb = static_cast<int>(K / 64);
-  g.rows = N;
-  g.cols = M;
-  g.k_total = K;
-  g.splits = p.s_main;
-  g.prof = 0;
-  // D[i = n, j = m] -> y[m, n]
-  return status_of(run_gemm(g, y, true, 1.0f, 1, N, N, M, M * N, part, d.err, cs));
+ql_status qlora_linear_fwd_w(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x, const ql_weight* w,
+                             const uint16_t* A, const uint16_t* B, float s, uint16_t* y, uint16_t* su_out,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  return linear_fwd_impl(M, N, K, r, x, w, A, B, s, y, su_out, workspace, ws_bytes, stream, nullptr);
 }
 
 ql_status qlora_linear_bwd(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* dy, const uint16_t* x,
                            const uint8_t* codes, const float* absmax, const uint16_t* A, const uint16_t* B, float s,
                            const uint16_t* su_in, uint16_t* dx, float* dA, float* dB, void* workspace, size_t ws_bytes,
                            void* stream) {
-  ql_status st = check_linear(M, N, K, r);
-  if (st != QL_OK) return st;
-  if (!codes || !absmax || !aligned16(codes) || !aligned16(absmax)) return QL_ERR_INVALID_ARG;
-  const bool want_da = r > 0 && dA, want_db = r > 0 && dB;
-  if ((dx && !aligned16(dx)) || (want_da && !aligned16(dA)) || (want_db && !aligned16(dB))) return QL_ERR_INVALID_ARG;
-  if (r > 0 && (!A || !B || !aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
-  if (su_in && !aligned16(su_in)) return QL_ERR_INVALID_ARG;
-  cudaStream_t cs = as_stream(stream);
-  if (M == 0) {
-    if (want_da && cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 4, cs) != cudaSuccess) return QL_ERR_CUDA;
-    if (want_db && cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 4, cs) != cudaSuccess) return QL_ERR_CUDA;
-    return QL_OK;
+  const ql_weight w = nf4_weight(codes, absmax);
+  return linear_bwd_impl(M, N, K, r, dy, x, &w, A, B, s, su_in, dx, dA, dB, workspace, ws_bytes, stream, nullptr);
+}
+
+ql_status qlora_linear_bwd_w(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* dy, const uint16_t* x,
+                             const ql_weight* w, const uint16_t* A, const uint16_t* B, float s, const uint16_t* su_in,
+                             uint16_t* dx, float* dA, float* dB, void* workspace, size_t ws_bytes, void* stream) {
+  return linear_bwd_impl(M, N, K, r, dy, x, w, A, B, s, su_in, dx, dA, dB, workspace, ws_bytes, stream, nullptr);
+}
+
+// Extra workspace of the gated calls: a dh buffer [M, F] bf16 when the down projection's dX GEMM splits its
+// contraction (the fused epilogue then cannot run, and dSwiGLU follows as its own kernel).
+size_t gated_dh_bytes(int64_t M, int64_t N, int64_t F, int64_t r) {
+  return plan_linear(M, N, F, r, QL_PASS_BWD).s_main > 1 ? align256(static_cast<size_t>(M) * F * 2) : 0;
+}
+
+size_t qlora_gated_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass) {
+  if (pass == QL_PASS_FWD) return qlora_workspace_bytes(M, N, K, r, pass);
+  const size_t base = align256(qlora_workspace_bytes(M, N, K, r, pass));
+  return M > 0 && check_linear(M, N, K, r) == QL_OK ? base + gated_dh_bytes(M, N, K, r) : 0;
+}
+
+ql_status qlora_gate_up_fwd_swiglu(int64_t M, int64_t F, int64_t K, int64_t r, const uint16_t* x, const uint8_t* codes,
+                                   const float* absmax, const uint16_t* A, const uint16_t* B, float s, uint16_t* gu,
+                                   uint16_t* h, uint16_t* su_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (F <= 0 || F % 16 != 0 || !h || !aligned16(h)) return QL_ERR_INVALID_ARG;
+  const int64_t N = 2 * F;
+  const ql_weight w = nf4_weight(codes, absmax);
+  if (check_linear(M, N, K, r) != QL_OK) return QL_ERR_INVALID_ARG;
+  // the fused epilogue runs in unsplit GEMMs with one-block stages; token-light layers (4-block stages) and
+  // split contractions write gu first and run the SwiGLU as its own kernel
+  if (M > 0 && plan_linear(M, N, K, r, QL_PASS_FWD).s_main == 1 && fwd_stage_blocks(M, K) == 1) {
+    EpiArgs e;
+    e.mode = EPI_SWIGLU_FWD;
+    e.out2 = h;
+    e.ls2 = 1;
+    e.cs2 = F;
+    return linear_fwd_impl(M, N, K, r, x, &w, A, B, s, gu, su_out, workspace, ws_bytes, stream, &e);
   }
-  if (!dy || !aligned16(dy)) return QL_ERR_INVALID_ARG;
-  if ((want_da || want_db || (r > 0 && !su_in)) && (!x || !aligned16(x))) return QL_ERR_INVALID_ARG;
-  const LinearPlan p = plan_linear(M, N, K, r, QL_PASS_BWD);
-  if (ws_bytes < p.total || (p.total > 0 && (!workspace || !aligned16(workspace)))) return QL_ERR_INVALID_ARG;
+  ql_status st = linear_fwd_impl(M, N, K, r, x, &w, A, B, s, gu, su_out, workspace, ws_bytes, stream, nullptr);
+  if (st != QL_OK || M == 0) return st;
   DeviceInfo d;
   if (!device_info(&d)) return QL_ERR_CUDA;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* part = ws ? reinterpret_cast<float*>(ws + p.off_part) : nullptr;
-  const int rp = rank_pad(r);
+  const long long groups = M * (F / 8);
+  const long long ctas = std::min<long long>(cdiv(groups, 256), static_cast<long long>(d.sms) * 16);
+  swiglu_interleaved_fwd_kernel<<<static_cast<unsigned>(ctas), 256, 0, as_stream(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(gu), reinterpret_cast<__nv_bfloat16*>(h), M, F);
+  count_launch();
+  return status_of(cudaGetLastError());
+}
 
-  uint16_t* v = nullptr;
-  const uint16_t* su = su_in;
-  if (r > 0) {
-    // su = bf16(s x A^T), recomputed when the forward's copy is not supplied (needed by dB)
-    if (!su && want_db) {
-      uint16_t* su_ws = reinterpret_cast<uint16_t*>(ws + p.off_su);
-      if (run_su(M, K, r, x, A, s, su_ws, p.s_su, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
-      su = su_ws;
-    }
-    // v = bf16(s dY B) [M, r]: D[i = m, j] = sum_n dY[m, n] B[n, j]
-    v = reinterpret_cast<uint16_t*>(ws + p.off_v);
-    GemmCall g;
-    g.am = A_TMA_K;
-    g.b_mn = true;
-    g.bn = rp;
-    g.a = {dy, M, N};
-    g.b = {B, N, r};
-    g.rows = M;
-    g.cols = rp;
-    g.k_total = N;
-    g.splits = p.s_v;
-    if (run_gemm(g, v, true, s, r, 1, M, r, M * r, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
+ql_status qlora_down_bwd_dswiglu(int64_t M, int64_t N, int64_t F, int64_t r, const uint16_t* dy, const uint16_t* h,
+                                 const uint8_t* codes, const float* absmax, const uint16_t* A, const uint16_t* B,
+                                 float s, const uint16_t* su, const uint16_t* gu, uint16_t* dgu, float* dA, float* dB,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  if (F <= 0 || F % 16 != 0 || !gu || !dgu || !aligned16(gu) || !aligned16(dgu)) return QL_ERR_INVALID_ARG;
+  const ql_weight w = nf4_weight(codes, absmax);
+  if (check_linear(M, N, F, r) != QL_OK) return QL_ERR_INVALID_ARG;
+  if (ws_bytes < qlora_gated_workspace_bytes(M, N, F, r, QL_PASS_BWD)) return QL_ERR_INVALID_ARG;
+  const size_t dh_bytes = M > 0 ? gated_dh_bytes(M, N, F, r) : 0;
+  if (dh_bytes == 0) {
+    EpiArgs e;
+    e.mode = EPI_DSWIGLU;
+    e.out2 = dgu;
+    e.aux = gu;
+    e.aux_ld = 2 * F;
+    // dx is only the switch that runs the dX GEMM: its epilogue writes dgu and never dx
+    return linear_bwd_impl(M, N, F, r, dy, h, &w, A, B, s, su, dgu, dA, dB, workspace, ws_bytes, stream, &e);
   }
-  if (dx) {
-    // dX^T: D[i = k, j = m] = sum_n deq(W)[n, k] dY[m, n]  (+ sum_j A[j, k] v[m, j])
-    GemmCall g;
-    g.am = A_DEQ_MN;
-    g.b_mn = false;
-    g.bn = p.bn_main;
-    g.b = {dy, M, N};
-    if (r > 0) {
-      // the LoRA rows: A extra = A [r, K] (copied into the MN-major tiles by the kernel), B extra = v
-      g.args.lora = A;
-      g.args.lora_ld = static_cast<int>(K);
-      g.args.lora_r = static_cast<int>(r);
-      g.bx = {v, M, r};
-      g.n_extra = static_cast<int>(cdiv(r, 64));
-    }
-    g.codes = codes;
-    g.args.absmax = absmax;
-    g.args.w_rows = static_cast<int>(N);
-    g.args.w_cols = static_cast<int>(K);
-    g.args.w_kb = static_cast<int>(K / 64);
-    g.rows = K;
-    g.cols = M;
-    g.k_total = N;
-    g.splits = p.s_main;
-    g.prof = 1;
-    if (run_gemm(g, dx, true, 1.0f, 1, K, K, M, M * K, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
-  }
-  if (want_da) {
-    // dA^T: D[i = k, j] = sum_m x[m, k] v[m, j]  -> dA[j, k]
-    GemmCall g;
-    g.am = A_TMA_MN;
-    g.b_mn = true;
-    g.bn = rp;
-    g.a = {x, M, K};
-    g.b = {v, M, r};
-    g.rows = K;
-    g.cols = rp;
-    g.k_total = M;
-    g.splits = p.s_da;
-    if (run_gemm(g, dA, false, 1.0f, 1, K, K, r, r * K, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
-  }
-  if (want_db) {
-    // dB: D[i = n, j] = sum_m dY[m, n] su[m, j]
-    GemmCall g;
-    g.am = A_TMA_MN;
-    g.b_mn = true;
-    g.bn = rp;
-    g.a = {dy, M, N};
-    g.b = {su, M, r};
-    g.rows = N;
-    g.cols = rp;
-    g.k_total = M;
-    g.splits = p.s_db;
-    if (run_gemm(g, dB, false, 1.0f, r, 1, N, r, N * r, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
-  }
-  return QL_OK;
+  // the layer's own workspace first, then the dh buffer (ws_bytes covers both, checked above)
+  if (!workspace || !aligned16(workspace)) return QL_ERR_INVALID_ARG;
+  const size_t base = align256(qlora_workspace_bytes(M, N, F, r, QL_PASS_BWD));
+  uint16_t* dh = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + base);
+  ql_status st = linear_bwd_impl(M, N, F, r, dy, h, &w, A, B, s, su, dh, dA, dB, workspace, base, stream, nullptr);
+  if (st != QL_OK) return st;
+  DeviceInfo d;
+  if (!device_info(&d)) return QL_ERR_CUDA;
+  const long long groups = M * (F / 8);
+  const long long ctas = std::min<long long>(cdiv(groups, 256), static_cast<long long>(d.sms) * 16);
+  swiglu_interleaved_bwd_kernel<<<static_cast<unsigned>(ctas), 256, 0, as_stream(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(dh), reinterpret_cast<const __nv_bfloat16*>(gu),
+      reinterpret_cast<__nv_bfloat16*>(dgu), M, F);
+  count_launch();
+  return status_of(cudaGetLastError());
 }
 
 ql_status qlora_merge_lora(int64_t N, int64_t K, int64_t r, const uint8_t* codes, const float* absmax,
@@ -752,23 +1154,71 @@ constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB on every devi
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-// Device address of g_noalloc_scratch per device.  In host code the array's name is only a host-side
-// stand-in, so the address is looked up once per device, with that device current.
-void* g_noalloc_ptr[kMaxDevices] = {};
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The calling thread's current context (driver entry point reached through the runtime), or nullptr.
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Loads every kernel the forward can launch, so that no later call in this context loads one lazily (a
+// module load may allocate).  cudaFuncGetAttributes forces the load and allocates nothing itself.
+template <int BN, int AM, bool BMN, int KB = 1, bool PAIR = false>
+bool load_umma() {
+  cudaFuncAttributes a;
+  return cudaFuncGetAttributes(&a, umma_gemm_kernel<BN, AM, BMN, KB, PAIR>) == cudaSuccess;
+}
+
+bool load_forward_kernels() {
+  cudaFuncAttributes a;
+  return load_umma<16, A_DEQ_TMEM, false>() && load_umma<32, A_DEQ_TMEM, false>() &&
+         load_umma<64, A_DEQ_TMEM, false>() && load_umma<128, A_DEQ_TMEM, false>() &&
+         load_umma<256, A_DEQ_TMEM, false>() && load_umma<256, A_DEQ_TMEM, false, 1, true>() &&
+         load_umma<16, A_DEQ_TMEM, false, 4>() &&
+         load_umma<32, A_DEQ_TMEM, false, 4>() && load_umma<64, A_DEQ_TMEM, false, 4>() &&
+         load_umma<64, A_TMA_K, false>() && load_umma<128, A_TMA_K, false>() && load_umma<256, A_TMA_K, false>() &&
+         cudaFuncGetAttributes(&a, reduce_splits_kernel) == cudaSuccess;
+}
+
+// Contexts in which the forward's kernels have been loaded (set-up runs once per context, with the device
+// current).
+CUcontext g_noalloc_ready[kMaxDevices * 4] = {};
+int g_noalloc_nready = 0;
 std::mutex g_noalloc_mu;
 
+// Device address of g_noalloc_scratch in the current context.  In host code the array's name is only a
+// host-side stand-in, so its address is looked up with the device current -- on every call, since it
+// belongs to the context (cudaDeviceReset or a non-primary context gives another one) and the lookup
+// allocates nothing once the module is loaded.  The first call in a context also loads the forward's
+// kernels.
 bool noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return false;
+  const CUcontext ctx = current_context();
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return false;
-    g_noalloc_ptr[dev] = p;
+  bool ready = false;
+  for (int i = 0; i < g_noalloc_nready && !ready; ++i) ready = (g_noalloc_ready[i] == ctx);
+  if (!ready) {
+    if (!load_forward_kernels()) return false;
+    if (ctx && g_noalloc_nready < kMaxDevices * 4) g_noalloc_ready[g_noalloc_nready++] = ctx;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = p;
   return true;
 }
+
 
 }  // namespace
 }  // namespace qlora

@@ -34,8 +34,9 @@
 //
 // Warp roles: warp 0 = B producer (lane 0 issues TMA), warp 1 = TMEM allocator + MMA issuer, warps 2..5 =
 // epilogue (TMEM -> registers -> global), warps 6 .. 6 + 4G - 1 = dequantizers (G groups of 4 warps; group
-// g % G takes stage g), warp 6 + 4G = Q producer (lane 0 issues the codes TMA, all lanes copy absmax).  The
-// dequantizer and Q-producer warps exist in the dequantizing modes only.
+// g % G takes stage g), warp 6 + 4G = Q producer (lane 0 issues the codes TMA, all lanes copy absmax), and in
+// the fused SwiGLU forward four more epilogue warps after it (each epilogue warp then drains half the
+// columns of its lane quarter).  The dequantizer and Q-producer warps exist in the dequantizing modes only.
 //
 // Shared-memory tiles: for the 128B swizzle every tile starts on a 1024-byte boundary; row r of a tile is
 // 128 bytes at r*128 and its 16-byte chunk c sits at chunk position c ^ (r & 7).  TMA writes that layout;
@@ -52,10 +53,34 @@
 
 #include "nf4_table.cuh"
 #include "ptx.cuh"
+#include "swiglu.cuh"
 
 namespace qlora {
 
-enum AMode : int { A_TMA_K = 0, A_TMA_MN = 1, A_DEQ_MN = 3, A_DEQ_TMEM = 4 };
+// A_DEQ_TMEM_T (backward dX): the transposed weight tile, dequantized straight into tensor memory -- each TMEM lane
+// (tile row = a column k of W) gathers its 64 contraction values from 64 rows of codes -- so the dX operand
+// needs no shared-memory round trip.  Codes and scales arrive as in A_DEQ_MN.
+enum AMode : int { A_TMA_K = 0, A_TMA_MN = 1, A_DEQ_MN = 3, A_DEQ_TMEM = 4, A_DEQ_TMEM_T = 5 };
+enum WFormat : int { WF_NF4 = 0, WF_NF4_DQ = 1, WF_NVFP4 = 2 };
+
+// E4M3 value of a finite pattern (sign bit 7, exponent bits 6..3 with bias 7, mantissa bits 2..0).
+__device__ __forceinline__ float e4m3_value_dev(uint32_t code) {
+  const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+  const float mag = e == 0 ? __fmul_rn(static_cast<float>(m), 0.001953125f) : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  return (code & 0x80u) ? -mag : mag;
+}
+
+// E2M1 value (sign bit 3, exponent bits 2..1 with bias 1, mantissa bit 0).
+__device__ __forceinline__ float e2m1_value_dev(uint32_t code) {
+  const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+  const float mag = e == 0 ? 0.5f * static_cast<float>(m) : static_cast<float>((2u + m) << (e - 1)) * 0.5f;
+  return (code & 8u) ? -mag : mag;
+}
+// Epilogue modes.  EPI_SWIGLU_FWD: the GEMM is the gate/up projection in the interleaved layout (gate_pos /
+// up_pos): besides gu = D it writes h = silu(g) * up to out2.  EPI_DSWIGLU: D is dh of a gated MLP's down
+// projection (rows = features): it reads g, up from aux (the saved gu) and writes dgu to out2 instead of dh.
+// Both need the whole contraction in one unit (no split) and bf16 outputs.
+enum Epi : int { EPI_PLAIN = 0, EPI_SWIGLU_FWD = 1, EPI_DSWIGLU = 2 };
 
 struct UmmaArgs {
   int rows, cols;         // D extent: i in [0, rows), j in [0, cols)
@@ -64,8 +89,18 @@ struct UmmaArgs {
   int k_stages;           // main contraction stages (64 KB elements each) in total
   int stages_per_split;   // main stages per split
   int n_extra;            // extra (LoRA) stages, run by split 0 only, before its main stages
-  // dequantization (A_DEQ_*): W is [w_rows, w_cols] with absmax [w_rows, w_cols / 64]
-  const float* absmax;
+  // dequantization (A_DEQ_*): W is [w_rows, w_cols] of packed 4-bit codes in format `wfmt` with one 4-byte
+  // scale word per 64-element block, `scale_words` [w_rows, w_cols / 64]:
+  //   WF_NF4    : the fp32 absmax of the block (codes: NF4 levels, element 2j in the high nibble);
+  //   WF_NF4_DQ : `scale_words` is the byte array of 8-bit double-quantized constants (one byte per block;
+  //               absmax = fl32(fl32(L[code] * dq_c1[block / 256]) + *dq_mu));
+  //   WF_NVFP4  : four E4M3 patterns, the scales of the block's four 16-element groups (decoded scale =
+  //               fl32(value * *fp4_S); codes: E2M1, element 2j in the low nibble).
+  const void* scale_words;
+  int wfmt;
+  const float* dq_c1;
+  const float* dq_mu;
+  const float* fp4_S;
   int w_rows, w_cols, w_kb;
   // LoRA matrix copied into the extra stages of A, row stride lora_ld, lora_r valid contraction entries:
   //   A_DEQ_TMEM: B [w_rows, lora_r] (tile row i = W row i0 + i, contraction along the row),
@@ -78,6 +113,20 @@ struct UmmaArgs {
   float alpha;
   long long ls, cs, split_stride;
   int rows_lim, cols_lim;
+  // fused epilogues (Epi): h [cols, rows / 2] at out2 + (row feature) * ls2 + j * cs2, or dgu at out2 with g, up
+  // read from aux, both [cols, 2 * rows] bf16 with row stride aux_ld
+  // cluster split-K (TMA modes): cred = S > 1 runs the S splits of one tile as the S CTAs of a cluster, which
+  // sum their fp32 partial tiles through distributed shared memory instead of writing slabs (0: off)
+  int cred;
+  // unit order: group_i > 0 walks the tiles in groups of group_i tile rows (weight tiles), tile rows fastest
+  // within a group, so that one wave of CTAs shares a few activation tiles and a group of weight tiles and
+  // both stay in L2; 0 keeps tile columns fastest
+  int group_i;
+  int epi;
+  void* out2;
+  long long ls2, cs2;
+  const uint16_t* aux;
+  long long aux_ld;
   unsigned int* err;
 };
 
@@ -86,14 +135,37 @@ struct Unit {
   int main_begin, n_main, n_extra, n_total;
 };
 
-// Unit u -> (split z, tile row ti, tile column tj), tj fastest: neighbouring units share the weight tile.
-__device__ __forceinline__ Unit unit_of(const UmmaArgs& a, int u, int BN) {
+// Unit u -> (split z, tile row ti, tile column tj).  Splits are outermost.  Within a split, either tile columns
+// run fastest (neighbouring units share the weight tile), or -- with group_i > 0 -- the tile rows come in groups
+// of group_i (the last group may be smaller) and within a group the rows run fastest: a wave of consecutive
+// units then covers group_i weight tiles and only a few activation tiles, so each is fetched from DRAM about
+// once per wave instead of the whole activation matrix being streamed again by every wave.
+// With CTA pairs a tile row is 256 weight rows and CTA `rank` of the pair owns rows 128 rank .. 128 rank + 127.
+__device__ __forceinline__ Unit unit_of(const UmmaArgs& a, int u, int BN, int pair = 1, int rank = 0) {
   Unit U;
-  const int tj = u % a.tiles_j;
-  const int t = u / a.tiles_j;
-  const int ti = t % a.tiles_i;
-  U.z = t / a.tiles_i;
-  U.i0 = ti * 128;
+  int tj, ti;
+  if (a.cred > 1) {  // the S consecutive units of a cluster are the S splits of one tile
+    U.z = u % a.cred;
+    const int t = u / a.cred;
+    tj = t % a.tiles_j;
+    ti = t / a.tiles_j;
+  } else if (a.group_i > 0) {
+    const int per_split = a.tiles_i * a.tiles_j;
+    U.z = u / per_split;
+    const int rem = u - U.z * per_split;
+    const int grp = rem / (a.group_i * a.tiles_j);
+    const int gi0 = grp * a.group_i;
+    const int gsz = a.tiles_i - gi0 < a.group_i ? a.tiles_i - gi0 : a.group_i;
+    const int local = rem - gi0 * a.tiles_j;
+    ti = gi0 + local % gsz;
+    tj = local / gsz;
+  } else {
+    tj = u % a.tiles_j;
+    const int t = u / a.tiles_j;
+    ti = t % a.tiles_i;
+    U.z = t / a.tiles_i;
+  }
+  U.i0 = ti * 128 * pair + 128 * rank;
   U.j0 = tj * BN;
   U.main_begin = U.z * a.stages_per_split;
   int end = U.main_begin + a.stages_per_split;
@@ -108,14 +180,18 @@ __device__ __forceinline__ Unit unit_of(const UmmaArgs& a, int u, int BN) {
 // barrier round trips of fixed latency, so token-light layers -- whose MMAs are short -- run 4 blocks a stage
 // (A_DEQ_TMEM only): codes then arrive as one 128B-swizzled TMA box of 128 rows x 128 bytes and the absmax
 // values as one TMA box of 128 rows x 4 floats.
-template <int BN, int AM, bool B_MN, int KB = 1>
+template <int BN, int AM, bool B_MN, int KB = 1, bool PAIR = false, int EPI = EPI_PLAIN>
 struct UmmaCfg {
-  static constexpr bool kATmem = (AM == A_DEQ_TMEM);
+  static constexpr int kPair = PAIR ? 2 : 1;   // CTAs per MMA (cta_group::2: M = 256)
+  static constexpr int kBRows = BN / kPair;    // B rows (tokens) held by each CTA
+  static constexpr bool kTrans = (AM == A_DEQ_TMEM_T);
+  static constexpr bool kATmem = (AM == A_DEQ_TMEM || kTrans);
+  static constexpr bool kQmn = (AM == A_DEQ_MN || kTrans);  // codes and scales in the MN-major slot layout
   static constexpr bool kDeq = (AM == A_DEQ_MN || kATmem);
   static constexpr bool kAMN = (AM == A_TMA_MN || AM == A_DEQ_MN);
   static constexpr bool kAbsTma = (KB == 4);  // absmax by TMA (else one cp.async per row)
   static constexpr int kTileA = 128 * 64 * 2;  // one bf16 A block in shared memory
-  static constexpr int kBBytes = BN * 64 * 2 * KB;
+  static constexpr int kBBytes = kBRows * 64 * 2 * KB;  // this CTA's share of a B stage
   static constexpr int kBSlot = kBBytes + (kDeq ? 0 : kTileA);  // the TMA modes load A beside B
   static constexpr int kASlot = (AM == A_DEQ_MN) ? kTileA : 0;   // A ring in shared memory
   static constexpr int kCBytes = 4096 * KB;                       // 128 rows x 64 KB codes
@@ -148,9 +224,15 @@ struct UmmaCfg {
   // spends most of a stage waiting on its own instruction latencies, so stage throughput grows with the
   // number of groups in flight, up to the A ring's depth: 4 in the TMEM kernel, 3 in the MN-major one.
   static constexpr int kDeqWarpsPerGroup = 4;
-  static constexpr int kDeqGroups = kDeq ? (kAStages < (kATmem ? 4 : 3) ? kAStages : (kATmem ? 4 : 3)) : 0;
+  // The fused SwiGLU forward epilogue is long and, with one accumulator at BN >= 128, not overlapped with the
+  // next unit's MMAs: it runs on 8 epilogue warps (two per lane quarter, each draining half the columns), and
+  // its CTA has one dequantizer group fewer to stay within the register file.
+  static constexpr int kEpiWarps = (EPI == EPI_SWIGLU_FWD && BN >= 128) ? 8 : 4;
+  static constexpr int kDeqCap = kATmem ? (kEpiWarps == 8 ? 3 : 4) : 3;
+  static constexpr int kDeqGroups = kDeq ? (kAStages < kDeqCap ? kAStages : kDeqCap) : 0;
   static constexpr int kQWarp = 6 + 4 * kDeqGroups;
-  static constexpr int kThreads = kDeq ? 32 * (kQWarp + 1) : 64 + 128;
+  // warps: producers and MMA (0, 1), epilogue (2..5), dequantizers, the Q producer, extra epilogue warps
+  static constexpr int kThreads = kDeq ? 32 * (kQWarp + 1 + kEpiWarps - 4) : 64 + 128;
   static constexpr int kTmemNeed = kAColBase + (kATmem ? kAStages * kAColsStage : 0);
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kSmemBytes =
@@ -159,7 +241,8 @@ struct UmmaCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is a multiple of 16 in [16, 256]");
   static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-element swizzle atoms");
   static_assert(!(kDeq && B_MN), "the dequantizing modes take B K-major");
-  static_assert(KB == 1 || (kATmem && KB == 4), "4-block stages exist for the TMEM forward only");
+  static_assert(KB == 1 || (AM == A_DEQ_TMEM && KB == 4), "4-block stages exist for the TMEM forward only");
+  static_assert(!PAIR || (kDeq && BN % 16 == 0), "CTA pairs: dequantizing modes, 8-row-aligned B halves");
   static_assert(kTmemNeed <= 512, "tensor memory");
   static_assert(kBStages >= 2 && (!kDeq || (kAStages >= 2 && kQStages >= 4)), "ring depths");
   // parity safety (see the kernel): Q ring deeper than the A ring by at least the number of dequantizer
@@ -197,12 +280,13 @@ struct Armed {
 };
 
 // tmA: A for the TMA modes; the absmax matrix [w_rows, w_cols / 64] (fp32) for 4-block TMEM stages.
-template <int BN, int AM, bool B_MN, int KB = 1>
-__global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
+template <int BN, int AM, bool B_MN, int KB = 1, bool PAIR = false, int WF = WF_NF4, int EPI = EPI_PLAIN>
+__global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC,
                      const UmmaArgs args) {
-  using C = UmmaCfg<BN, AM, B_MN, KB>;
+  using C = UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>;
+  static_assert(AM != A_DEQ_TMEM_T || WF == WF_NF4, "the transposed TMEM dequantizer reads NF4 weights");
   constexpr int BS = C::kBStages;
   constexpr int AS = C::kAStages;
   constexpr int QS = C::kQStages;
@@ -240,6 +324,11 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_units = args.splits * args.tiles_i * args.tiles_j;
+  // CTA pairs: the even CTA of the cluster (rank 0) is the leader -- it issues the pair's MMAs, and its barriers
+  // gather both CTAs' arrivals; each pair walks the units together
+  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const int first_unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int unit_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < BS; ++s) {
@@ -247,26 +336,29 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
       mbar_init(&b_empty[s], 1);
     }
     for (int s = 0; s < AS; ++s) {
-      mbar_init(&a_full[s], C::kDeqWarpsPerGroup);
+      mbar_init(&a_full[s], C::kDeqWarpsPerGroup * C::kPair);
       mbar_init(&a_empty[s], 1);
     }
     for (int s = 0; s < QS; ++s) {
-      mbar_init(&q_full[s], C::kAbsTma ? 1 : 1 + 32);  // the TMA arrive (+ one cp.async arrive per producer lane)
+      // the TMA arrive (+ one cp.async arrive per producer lane when the scale words come by cp.async)
+      mbar_init(&q_full[s], C::kAbsTma && WF != WF_NF4_DQ ? 1 : 1 + 32);
       mbar_init(&q_empty[s], C::kDeqWarpsPerGroup * 32);  // every lane of the consuming group
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], 4);
+      mbar_init(&tmem_empty[b], C::kEpiWarps * C::kPair);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   if constexpr (C::kLutBytes > 0) {
-    // entry (byte b, lane l) at word 32 b + l: the bf16 pair (level[b >> 4], level[b & 15]) -- a code byte
-    // holds element 2j in its high nibble, and the first element goes to the low half
+    // entry (byte b, lane l) at word 32 b + l: the bf16 pair of the byte's two elements, element 2j in the low
+    // half.  NF4 bytes hold element 2j in the high nibble, NVFP4 bytes in the low nibble.
+    constexpr bool fp4 = WF == WF_NVFP4;
     for (int idx = threadIdx.x; idx < 256 * 32; idx += blockDim.x) {
       const int b = idx >> 5;
-      __nv_bfloat162 h = __floats2bfloat162_rn(kNF4LevelsDev[b >> 4], kNF4LevelsDev[b & 15]);
+      __nv_bfloat162 h = fp4 ? __floats2bfloat162_rn(e2m1_value_dev(b & 15), e2m1_value_dev(b >> 4))
+                             : __floats2bfloat162_rn(kNF4LevelsDev[b >> 4], kNF4LevelsDev[b & 15]);
       sLut[idx] = *reinterpret_cast<uint32_t*>(&h);
     }
   }
@@ -277,14 +369,20 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
   }
   if (C::kDeq && warp == C::kQWarp && lane == 0) {
     tma_prefetch_desc(&tmC);
-    if (C::kAbsTma) tma_prefetch_desc(&tmA);
+    if (C::kAbsTma && WF != WF_NF4_DQ) tma_prefetch_desc(&tmA);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // the peer arrives on our barriers only once they exist
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -293,8 +391,8 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
     Armed armed;
     int g = 0;
     bool stop = false;
-    for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
-      const Unit U = unit_of(args, u, BN);
+    for (int u = first_unit; u < num_units && !stop; u += unit_step) {
+      const Unit U = unit_of(args, u, BN, C::kPair, rank);
       for (int it = 0; it < U.n_total; ++it, ++g) {
         const int s = g % BS;
         const uint32_t ph = static_cast<uint32_t>(g / BS) & 1u;
@@ -307,15 +405,19 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
           armed.set(s, ph);
           uint8_t* b_dst = sB + s * C::kBSlot;
           if constexpr (C::kDeq) {
-            // KB blocks of BN x 64, each a 128B-swizzled K-major sub-tile
-            mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
+            // KB blocks of kBRows x 64 (this CTA's share of the BN tokens), each a 128B-swizzled K-major
+            // sub-tile; with CTA pairs both halves complete on the leader's barrier, which expects both
+            if (rank == 0) mbar_arrive_expect_tx(&b_full[s], C::kPair * C::kBBytes);
+            const int jb = U.j0 + rank * C::kBRows;
 #pragma unroll
             for (int kb = 0; kb < KB; ++kb) {
-              if (it < U.n_extra)
-                tma_load_2d(b_dst + kb * BN * 128, &tmBx, 64 * (KB * it + kb), U.j0, &b_full[s]);
+              uint8_t* dst = b_dst + kb * C::kBRows * 128;
+              const int x = it < U.n_extra ? 64 * (KB * it + kb) : ((U.main_begin + it - U.n_extra) * KB + kb) * 64;
+              const CUtensorMap* tm = it < U.n_extra ? &tmBx : &tmB;
+              if constexpr (PAIR)
+                tma_load_2d_pair(dst, tm, x, jb, &b_full[s]);
               else
-                tma_load_2d(b_dst + kb * BN * 128, &tmB, ((U.main_begin + it - U.n_extra) * KB + kb) * 64, U.j0,
-                            &b_full[s]);
+                tma_load_2d(dst, tm, x, jb, &b_full[s]);
             }
           } else {
             // the TMA modes have no extra stages
@@ -338,19 +440,27 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
         }
       }
     }
-    // copies still in flight must land before the CTA's shared memory is released
-    if (lane == 0 && *abort_flag) armed.drain(b_full, BS, args.err);
+    // copies still in flight must land before the CTA's shared memory is released (a pair's copies complete
+    // on the leader's barriers: the leader drains them, and the closing cluster barrier holds the follower)
+    if (lane == 0 && *abort_flag && rank == 0) armed.drain(b_full, BS, args.err);
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (whole warp waits,
     // one elected lane issues)
-    constexpr uint32_t idesc = idesc_bf16_f32(128, BN, C::kAMN, B_MN);
+    constexpr uint32_t idesc = idesc_bf16_f32(PAIR ? 256 : 128, BN, C::kAMN, B_MN);
+    // barriers the peer CTA also arrives on are waited with acquire at cluster scope
+    auto wait_mma = [&](uint64_t* bar, uint32_t par) {
+      if constexpr (PAIR)
+        return mbar_wait_cluster(bar, par, abort_flag, args.err);
+      else
+        return mbar_wait(bar, par, abort_flag, args.err);
+    };
     int g = 0, lu = 0;
-    bool stop = false;
-    for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x, ++lu) {
-      const Unit U = unit_of(args, u, BN);
+    bool stop = rank != 0;  // the pair's follower issues nothing
+    for (int u = first_unit; u < num_units && !stop; u += unit_step, ++lu) {
+      const Unit U = unit_of(args, u, BN, C::kPair, rank);
       const int acc = lu % C::kAccBufs;
       const uint32_t eph = (static_cast<uint32_t>(lu / C::kAccBufs) & 1u) ^ 1u;
-      if (!__all_sync(kFull, mbar_wait(&tmem_empty[acc], eph, abort_flag, args.err))) break;
+      if (!__all_sync(kFull, wait_mma(&tmem_empty[acc], eph))) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccCols);
       for (int it = 0; it < U.n_total; ++it, ++g) {
@@ -359,8 +469,8 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
         bool ok;
         if constexpr (C::kDeq) {
           as = g % AS;
-          ok = mbar_wait(&a_full[as], static_cast<uint32_t>(g / AS) & 1u, abort_flag, args.err) &&
-               mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err);
+          ok = wait_mma(&a_full[as], static_cast<uint32_t>(g / AS) & 1u) &&
+               wait_mma(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u);
         } else {
           ok = mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err);
         }
@@ -375,33 +485,52 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4 * KB; ++kk) {
             const int kb = kk >> 2, k = kk & 3;
-            const uint32_t bk = b0 + static_cast<uint32_t>(kb * BN * 128);
+            const uint32_t bk = b0 + static_cast<uint32_t>(kb * C::kBRows * 128);
             const uint64_t bdesc = B_MN ? sdesc_sw128(bk + k * 2048, 8192, 1024) : sdesc_sw128(bk + k * 32, 16, 1024);
             const uint32_t accum = (it > 0 || kk > 0) ? 1u : 0u;
             if constexpr (C::kATmem) {
               const uint32_t a_tmem =
                   tmem_base + static_cast<uint32_t>(C::kAColBase + as * C::kAColsStage + kb * 32 + k * 8);
-              umma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, accum);
+              if constexpr (PAIR)
+                umma_bf16_ts_pair(d_tmem, a_tmem, bdesc, idesc, accum);
+              else
+                umma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, accum);
             } else {
               const uint64_t adesc =
                   C::kAMN ? sdesc_sw128(a0 + k * 2048, 8192, 1024) : sdesc_sw128(a0 + k * 32, 16, 1024);
-              umma_bf16_ss(d_tmem, adesc, bdesc, idesc, accum);
+              if constexpr (PAIR)
+                umma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, accum);
+              else
+                umma_bf16_ss(d_tmem, adesc, bdesc, idesc, accum);
             }
           }
-          umma_commit(&b_empty[bs]);
-          if constexpr (C::kDeq) umma_commit(&a_empty[as]);
+          if constexpr (PAIR) {  // the commits arrive on the barrier at this offset in both CTAs
+            umma_commit_pair(&b_empty[bs]);
+            umma_commit_pair(&a_empty[as]);
+          } else {
+            umma_commit(&b_empty[bs]);
+            if constexpr (C::kDeq) umma_commit(&a_empty[as]);
+          }
         }
         __syncwarp();
       }
-      if (elect_one()) umma_commit(&tmem_full[acc]);  // also on abort, so the MMAs issued can be waited for
+      if (elect_one()) {  // also on abort, so the MMAs issued can be waited for
+        if constexpr (PAIR)
+          umma_commit_pair(&tmem_full[acc]);
+        else
+          umma_commit(&tmem_full[acc]);
+      }
       __syncwarp();
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------------ epilogue (warps 2..5)
+  } else if (warp < 6 || warp > C::kQWarp) {
+    // ------------------------------------------------------------------ epilogue (warps 2..5, and with 8
+    // epilogue warps also the last four: those drain the second half of the columns)
     const int qw = warp & 3;  // TMEM lane quarter this warp may access
+    constexpr int kCols = BN * 4 / C::kEpiWarps;
+    const int c_begin = warp < 6 ? 0 : kCols, c_end = c_begin + kCols;
     int lu = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++lu) {
-      const Unit U = unit_of(args, u, BN);
+    for (int u = first_unit; u < num_units; u += unit_step, ++lu) {
+      const Unit U = unit_of(args, u, BN, C::kPair, rank);
       const int acc = lu % C::kAccBufs;
       int ok = mbar_wait_idle(&tmem_full[acc], static_cast<uint32_t>(lu / C::kAccBufs) & 1u, abort_flag, args.err) ? 1 : 0;
       tc_fence_after();
@@ -410,12 +539,91 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
       const int i = U.i0 + qw * 32 + lane;
       const long long base = static_cast<long long>(U.z) * args.split_stride + static_cast<long long>(i) * args.ls;
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + static_cast<uint32_t>(acc * C::kAccCols);
+      // EPI_DSWIGLU: g (low half) and up (high half) of this row's feature for the 16 tokens of the next chunk
+      // (tokens past the count read the last token's row: in bounds, never stored)
+      uint32_t gunext[EPI == EPI_DSWIGLU ? 16 : 1];
+      auto load_gu = [&](int cc, long long pg) {
+        if constexpr (EPI == EPI_DSWIGLU) {
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = min(U.j0 + cc + jj, args.cols_lim - 1);
+            const uint16_t* row = args.aux + static_cast<long long>(j) * args.aux_ld;
+            gunext[jj] = static_cast<uint32_t>(__ldg(row + pg)) | (static_cast<uint32_t>(__ldg(row + pg + 16)) << 16);
+          }
+        }
+      };
+      if constexpr (EPI == EPI_DSWIGLU) load_gu(c_begin, gate_pos(i < args.rows_lim ? i : 0));
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
+      for (int c0 = c_begin; c0 < c_end; c0 += 16) {
         uint32_t r[16];
         __syncwarp();  // tcgen05.ld is warp-aligned: reconverge after the guarded stores
         tmem_ld_32x32b_x16(t_acc + static_cast<uint32_t>(c0), r);
         tmem_ld_wait();
+        if (!C::kDeq && args.cred > 1) {
+          // this split's raw fp32 partial of the tile, row i - i0, parked in the (drained) B ring
+          float* prow = reinterpret_cast<float*>(sB) + (qw * 32 + lane) * (BN + 4) + c0;
+#pragma unroll
+          for (int jj = 0; jj < 16; jj += 4)
+            *reinterpret_cast<float4*>(prow + jj) =
+                U.n_total > 0 ? make_float4(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1]),
+                                            __uint_as_float(r[jj + 2]), __uint_as_float(r[jj + 3]))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          continue;
+        }
+        if constexpr (EPI == EPI_SWIGLU_FWD) {
+          // gu as stored (bf16); lanes l and l ^ 16 hold g and up of one feature.  Each lane of the pair forms
+          // h for half of the chunk's tokens -- the gate lane the even ones, the up lane the odd ones -- so all
+          // lanes do the same work
+          const bool gate = (lane & 16) == 0;
+          const long long feat = static_cast<long long>(i >> 5) * 16 + (lane & 15);
+          float v[16], pv[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = U.j0 + c0 + jj;
+            const __nv_bfloat16 b = __float2bfloat16_rn(U.n_total > 0 ? args.alpha * __uint_as_float(r[jj]) : 0.0f);
+            v[jj] = __bfloat162float(b);
+            if (i < args.rows_lim && j < args.cols_lim)
+              reinterpret_cast<__nv_bfloat16*>(args.out)[base + static_cast<long long>(j) * args.cs] = b;
+          }
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) pv[jj] = __shfl_xor_sync(kFull, v[jj], 16);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float g = gate ? v[2 * t] : pv[2 * t + 1];
+            const float u = gate ? pv[2 * t] : v[2 * t + 1];
+            const int j = U.j0 + c0 + 2 * t + (gate ? 0 : 1);
+            if (i < args.rows_lim && j < args.cols_lim)
+              reinterpret_cast<__nv_bfloat16*>(args.out2)[feat * args.ls2 + static_cast<long long>(j) * args.cs2] =
+                  __float2bfloat16_rn(swiglu_h(g, u));
+          }
+          continue;
+        }
+        if constexpr (EPI == EPI_DSWIGLU) {
+          // dh as stored (bf16), with g and up of feature i from the saved gu, gives the two halves of dgu.  The
+          // chunk's g and up were loaded one chunk ahead (dgu stores may alias gu as far as the compiler knows,
+          // so it would not hoist the loads itself)
+          const long long pg = gate_pos(i < args.rows_lim ? i : 0), pu = pg + 16;
+          uint32_t gucur[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) gucur[jj] = gunext[jj];
+          if (c0 + 16 < c_end) load_gu(c0 + 16, pg);
+          if (i < args.rows_lim) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = U.j0 + c0 + jj;
+              if (j < args.cols_lim) {
+                const float d = __bfloat162float(
+                    __float2bfloat16_rn(U.n_total > 0 ? args.alpha * __uint_as_float(r[jj]) : 0.0f));
+                float dg, du;
+                swiglu_grads(d, __uint_as_float(gucur[jj] << 16), __uint_as_float(gucur[jj] & 0xFFFF0000u), dg, du);
+                __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(args.out2) + static_cast<long long>(j) * args.aux_ld;
+                o[pg] = __float2bfloat16_rn(dg);
+                o[pu] = __float2bfloat16_rn(du);
+              }
+            }
+          }
+          continue;
+        }
         if (i < args.rows_lim) {
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
@@ -433,7 +641,12 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_leader(&tmem_empty[acc]);
+        else
+          mbar_arrive(&tmem_empty[acc]);
+      }
     }
   } else if (warp == C::kQWarp) {
     // ------------------------------------------------------------------ Q producer (dequantizing modes)
@@ -441,8 +654,8 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
       Armed armed;
       int q = 0;
       bool stop = false;
-      for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
-        const Unit U = unit_of(args, u, BN);
+      for (int u = first_unit; u < num_units && !stop; u += unit_step) {
+        const Unit U = unit_of(args, u, BN, C::kPair, rank);
         for (int it = U.n_extra; it < U.n_total; ++it, ++q) {
           const int s = q % QS;
           const uint32_t ph = static_cast<uint32_t>(q / QS) & 1u;
@@ -453,37 +666,49 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
           }
           const int kk0 = (U.main_begin + it - U.n_extra) * 64 * KB;
           uint8_t* q_dst = sQ + s * C::kQSlot;
+          // 4-block stages take their scale words by TMA, except the double-quantized constants (4 bytes a row,
+          // below the 16-byte minimum of a TMA box row)
+          constexpr bool scale_tma = C::kAbsTma && WF != WF_NF4_DQ;
           if (lane == 0) {
             armed.set(s, ph);
-            if constexpr (C::kAbsTma) {
-              // 128 W rows x 128 bytes of codes (swizzled) and 128 rows x 4 absmax values
+            if constexpr (scale_tma) {
+              // 128 W rows x 128 bytes of codes (swizzled) and 128 rows x 4 scale words
               mbar_arrive_expect_tx(&q_full[s], C::kCBytes + C::kSBytes);
               tma_load_2d(q_dst, &tmC, kk0 / 2, U.i0, &q_full[s]);
-              tma_load_2d(q_dst + C::kCBytes, &tmA, kk0 / 64, U.i0, &q_full[s]);
+              tma_load_2d(q_dst + C::kCBytes, &tmA, WF == WF_NVFP4 ? kk0 / 16 : kk0 / 64, U.i0, &q_full[s]);
+            } else if constexpr (C::kAbsTma) {
+              mbar_arrive_expect_tx(&q_full[s], C::kCBytes);
+              tma_load_2d(q_dst, &tmC, kk0 / 2, U.i0, &q_full[s]);
             } else {
               mbar_arrive_expect_tx(&q_full[s], C::kCBytes);
-              if constexpr (AM == A_DEQ_TMEM)
+              if constexpr (!C::kQmn)
                 tma_load_2d(q_dst, &tmC, kk0 / 2, U.i0, &q_full[s]);  // 128 W rows x 32 bytes
               else
                 tma_load_2d(q_dst, &tmC, U.i0 / 2, kk0, &q_full[s]);  // 64 W rows x 64 bytes
             }
           }
-          if constexpr (C::kAbsTma) continue;
-          float* sdst = reinterpret_cast<float*>(q_dst + C::kCBytes);
+          if constexpr (scale_tma) continue;
+          // one 4-byte word per (row, block): the fp32 absmax or the four NVFP4 group scales of the block; for
+          // the double-quantized constants the aligned word holding the block's byte (with 4-block stages, the
+          // word of the stage's four bytes, stored at the row's 16-byte scale slot)
+          uint32_t* sdst = reinterpret_cast<uint32_t*>(q_dst + C::kCBytes);
+          const uint8_t* words8 = static_cast<const uint8_t*>(args.scale_words);
+          constexpr bool dq = WF == WF_NF4_DQ;
 #pragma unroll
           for (int qq = 0; qq < 4; ++qq) {
             const int idx = lane + 32 * qq;
             int n, k;
-            if constexpr (AM == A_DEQ_TMEM) {  // value for tile row idx (W row i0 + idx) in k-block kk0 / 64
+            if constexpr (!C::kQmn) {  // word for tile row idx (W row i0 + idx) in k-block kk0 / 64
               n = U.i0 + idx;
               k = kk0;
-            } else {                           // value for W row kk0 + idx / 2 in k-block (i0 + 64 (idx & 1)) / 64
+            } else {                           // word for W row kk0 + idx / 2 in k-block (i0 + 64 (idx & 1)) / 64
               n = kk0 + (idx >> 1);
               k = U.i0 + 64 * (idx & 1);
             }
             const bool valid = n < args.w_rows && k < args.w_cols;
-            const float* src = valid ? args.absmax + static_cast<long long>(n) * args.w_kb + (k >> 6) : args.absmax;
-            cp_async_4_zfill(sdst + idx, src, valid);
+            const long long blk = static_cast<long long>(n) * args.w_kb + (k >> 6);
+            const uint8_t* src = !valid ? words8 : dq ? words8 + (blk & ~3ll) : words8 + 4 * blk;
+            cp_async_4_zfill(sdst + (C::kAbsTma ? 4 * idx : idx), src, valid);
           }
           cp_async_mbar_arrive_noinc(&q_full[s]);
         }
@@ -505,19 +730,23 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
       const int s_idx = C::kATmem ? row : (row * 2 + h);
       const uint32_t t_lane = static_cast<uint32_t>(32 * (warp & 3)) << 16;
       const uint8_t* lut_lane = reinterpret_cast<const uint8_t*>(sLut) + lane * 4;
+      const float dq_mu = WF == WF_NF4_DQ ? *args.dq_mu : 0.0f;
+      const float fp4_S = WF == WF_NVFP4 ? *args.fp4_S : 0.0f;
       int g = 0, q = 0;
       bool stop = false;
-      for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
-        const Unit U = unit_of(args, u, BN);
+      for (int u = first_unit; u < num_units && !stop; u += unit_step) {
+        const Unit U = unit_of(args, u, BN, C::kPair, rank);
         for (int it = 0; it < U.n_total; ++it, ++g) {
           const bool extra = it < U.n_extra;
           const int qi = q;
           if (!extra) ++q;
           if (g % C::kDeqGroups != grp) continue;
           // The stage's codes and scales, held in registers: block p of the stage is words[8p .. 8p + 7]
-          // (64 codes) with scale sc[p].
+          // (64 codes) with scale word sw[p] (for the double-quantized constants: the aligned word that holds
+          // the block's byte, or with 4-block stages the stage's four bytes, in sw[0]).
           uint32_t words[8 * KB];
-          float sc[KB];
+          uint32_t sw[KB] = {};  // (the transposing dequantizer reads its scales straight from the slot)
+          uint32_t r[32];  // the stage's 64 bf16 values (the first block's), packed in pairs
           if (!extra) {
             const int qs = qi % QS;
             const bool okq = mbar_wait_idle(&q_full[qs], static_cast<uint32_t>(qi / QS) & 1u, abort_flag, args.err);
@@ -526,7 +755,23 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
               break;
             }
             const uint8_t* q_src = sQ + qs * C::kQSlot;
-            if constexpr (C::kAbsTma) {
+            if constexpr (C::kTrans) {
+              // tile row `row` = column k = i0 + row of W: its code in each of the stage's 64 W rows is byte
+              // row / 2 of the row's 64 (the high nibble for even k), its scale that of the row's k-block
+              // (i0 + 64 (row / 64)) / 64; two rows per pair lookup, two scales per bf16x2 product
+              const uint8_t* cb = q_src + (row >> 1);
+              const float* sb = reinterpret_cast<const float*>(q_src + C::kCBytes) + (row >> 6);
+              const uint32_t sh = (row & 1) ? 0u : 4u;
+#pragma unroll
+              for (int pp = 0; pp < 32; ++pp) {
+                const uint32_t c0 = (static_cast<uint32_t>(cb[(2 * pp) * 64]) >> sh) & 15u;
+                const uint32_t c1 = (static_cast<uint32_t>(cb[(2 * pp + 1) * 64]) >> sh) & 15u;
+                uint32_t v = *reinterpret_cast<const uint32_t*>(lut_lane + (((c0 << 4) | c1) << 7));
+                const __nv_bfloat162 s2 = __floats2bfloat162_rn(sb[(2 * pp) * 2], sb[(2 * pp + 1) * 2]);
+                const __nv_bfloat162 pr = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), s2);
+                r[pp] = *reinterpret_cast<const uint32_t*>(&pr);
+              }
+            } else if constexpr (C::kAbsTma) {
               // row `row` is 128 bytes; its 16-byte chunk c sits at chunk position c ^ (row & 7)
               const uint8_t* q_row = q_src + row * 128;
 #pragma unroll
@@ -537,15 +782,15 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
                 words[4 * c + 2] = v.z;
                 words[4 * c + 3] = v.w;
               }
-              const float4 s4 = *reinterpret_cast<const float4*>(q_src + C::kCBytes + row * 16);
-              sc[0] = s4.x;
+              const uint4 s4 = *reinterpret_cast<const uint4*>(q_src + C::kCBytes + row * 16);
+              sw[0] = s4.x;
               if constexpr (KB == 4) {
-                sc[1] = s4.y;
-                sc[2] = s4.z;
-                sc[3] = s4.w;
+                sw[1] = s4.y;
+                sw[2] = s4.z;
+                sw[3] = s4.w;
               }
             } else {
-              sc[0] = reinterpret_cast<const float*>(q_src + C::kCBytes)[s_idx];
+              sw[0] = reinterpret_cast<const uint32_t*>(q_src + C::kCBytes)[s_idx];
               const uint4 c01 = *reinterpret_cast<const uint4*>(q_src + c_off);
               const uint4 c23 = *reinterpret_cast<const uint4*>(q_src + c_off + 16);
               words[0] = c01.x;
@@ -591,10 +836,38 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
                 r[4 * c + 3] = v.w;
               }
             } else {
-              // level pair from this lane's copy of the table, times the block scale in bf16x2
-              const __nv_bfloat162 sc2 = __float2bfloat162_rn(sc[p]);
+              // level pair from this lane's copy of the table, times the scale of its 16-element group in bf16x2
+              __nv_bfloat162 sc2q[4];
+              if constexpr (WF == WF_NVFP4) {
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq)
+                  sc2q[gq] = __float2bfloat162_rn(__fmul_rn(e4m3_value_dev((sw[p] >> (8 * gq)) & 0xFFu), fp4_S));
+              } else {
+                float a;
+                if constexpr (WF == WF_NF4_DQ) {
+                  // this thread's W row and k-block of block p (the producer's word holds its byte)
+                  int n, kb;
+                  if constexpr (C::kATmem) {
+                    n = U.i0 + row;
+                    kb = (U.main_begin + it - U.n_extra) * KB + p;
+                  } else {
+                    n = (U.main_begin + it - U.n_extra) * 64 + row;
+                    kb = (U.i0 >> 6) + h;
+                  }
+                  const long long blk = static_cast<long long>(n) * args.w_kb + kb;
+                  const uint32_t code = (sw[KB == 4 ? 0 : p] >> (8 * static_cast<int>(blk & 3))) & 0xFFu;
+                  a = (n < args.w_rows && kb < args.w_kb)
+                          ? __fadd_rn(__fmul_rn(__fdiv_rn(e4m3_value_dev(code), 448.0f), __ldg(args.dq_c1 + (blk >> 8))),
+                                      dq_mu)
+                          : 0.0f;
+                } else {
+                  a = __uint_as_float(sw[p]);
+                }
+                sc2q[0] = sc2q[1] = sc2q[2] = sc2q[3] = __float2bfloat162_rn(a);
+              }
 #pragma unroll
               for (int w = 0; w < 8; ++w) {
+                const __nv_bfloat162 sc2 = sc2q[w >> 1];
                 const uint32_t qw8 = words[8 * p + w];
                 const uint32_t offs[4] = {(qw8 << 7) & 0x7F80u, (qw8 >> 1) & 0x7F80u, (qw8 >> 9) & 0x7F80u,
                                           (qw8 >> 17) & 0x7F80u};
@@ -607,8 +880,24 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
               }
             }
           };
-          uint32_t r[32];
-          block_values(0, r);
+          if constexpr (C::kTrans) {
+            if (extra) {
+              // LoRA rows of A [lora_r, w_cols]: tile row k = i0 + row takes column k of the stage's 64 rows
+              const int k = U.i0 + row;
+              const bool vk = k < args.w_cols;
+#pragma unroll
+              for (int pp = 0; pp < 32; ++pp) {
+                const int j = 64 * it + 2 * pp;
+                const uint32_t lo = (vk && j < args.lora_r)
+                                        ? __ldg(args.lora + static_cast<long long>(j) * args.lora_ld + k) : 0u;
+                const uint32_t hi = (vk && j + 1 < args.lora_r)
+                                        ? __ldg(args.lora + static_cast<long long>(j + 1) * args.lora_ld + k) : 0u;
+                r[pp] = lo | (hi << 16);
+              }
+            }
+          } else {
+            block_values(0, r);
+          }
           // the A slot is free once the MMAs of its previous stage have completed
           const int as = g % AS;
           const bool oka = mbar_wait_idle(&a_empty[as], (static_cast<uint32_t>(g / AS) & 1u) ^ 1u, abort_flag, args.err);
@@ -619,7 +908,12 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
           tc_fence_after();
           // the MMAs of the slot's previous stage read it through the async proxy; order those reads before
           // this thread's generic writes
-          if constexpr (!C::kATmem) fence_proxy_async_smem();
+          if constexpr (!C::kATmem) {
+            if constexpr (PAIR)
+              fence_proxy_async_smem_cluster();
+            else
+              fence_proxy_async_smem();
+          }
           if constexpr (C::kATmem) {
             const uint32_t a_col = tmem_base + t_lane + static_cast<uint32_t>(C::kAColBase + as * C::kAColsStage);
             tmem_st_32x32b_x32(a_col, r);
@@ -636,11 +930,18 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
             for (int w = 0; w < 8; ++w)
               *reinterpret_cast<uint4*>(a_row + ((w ^ (row & 7)) << 4)) =
                   make_uint4(r[4 * w], r[4 * w + 1], r[4 * w + 2], r[4 * w + 3]);
-            fence_proxy_async_smem();
+            // visible to the async proxy -- with CTA pairs, to the leader's MMA reading this CTA's tile
+            if constexpr (PAIR)
+              fence_proxy_async_smem_cluster();
+            else
+              fence_proxy_async_smem();
           }
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&a_full[as]);  // the warp's quarter of the A stage is in place
+          if (lane == 0) {  // this warp's quarter of the A stage is in place (with pairs: on the leader's barrier)
+            if constexpr (PAIR)
+              mbar_arrive_leader(&a_full[as]);
+            else
+              mbar_arrive(&a_full[as]);
           }
           stop = __shfl_sync(kFull, stop ? 1 : 0, 0) != 0;
           if (stop) break;
@@ -651,10 +952,61 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair stays together to the end: the peer may still arrive on our barriers or have copies in flight
+  // counted on the leader's, and tensor memory is released by both CTAs together
+  if constexpr (PAIR) cluster_sync_all();
+  if constexpr (!C::kDeq && !PAIR) {
+    if (args.cred > 1) {
+      // cluster split-K: every CTA holds one split's partial tile (one unit each); CTA c sums rows
+      // [c R, (c + 1) R) of the tile over the S partials in split order -- the order of the slab reduction --
+      // then scales and stores them.  The second barrier keeps every CTA's shared memory alive until read.
+      cluster_sync_all();
+      const int S = args.cred;
+      const int c = static_cast<int>(cluster_ctarank());
+      const Unit U = unit_of(args, static_cast<int>(blockIdx.x), BN);
+      const int R = 128 / S;
+      const int per_row = BN / 4;
+      const uint32_t base_addr = smem_u32(sB);
+      if (warp >= 2 && warp < 6) {
+        for (int e = threadIdx.x - 64; e < R * per_row; e += 128) {
+          const int row = c * R + e / per_row, col = (e % per_row) * 4;
+          const uint32_t off = static_cast<uint32_t>((row * (BN + 4) + col) * 4);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int src = 0; src < S; ++src) {
+            const float4 v = ld_dsmem_f32x4(mapa_cluster(base_addr + off, static_cast<uint32_t>(src)));
+            acc.x = __fadd_rn(acc.x, v.x);
+            acc.y = __fadd_rn(acc.y, v.y);
+            acc.z = __fadd_rn(acc.z, v.z);
+            acc.w = __fadd_rn(acc.w, v.w);
+          }
+          const int i = U.i0 + row;
+          if (i < args.rows_lim) {
+            const float o[4] = {__fmul_rn(acc.x, args.alpha), __fmul_rn(acc.y, args.alpha),
+                                __fmul_rn(acc.z, args.alpha), __fmul_rn(acc.w, args.alpha)};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int j = U.j0 + col + q;
+              if (j < args.cols_lim) {
+                const long long at = static_cast<long long>(i) * args.ls + static_cast<long long>(j) * args.cs;
+                if (args.out_bf16)
+                  reinterpret_cast<__nv_bfloat16*>(args.out)[at] = __float2bfloat16_rn(o[q]);
+                else
+                  reinterpret_cast<float*>(args.out)[at] = o[q];
+              }
+            }
+          }
+        }
+      }
+      cluster_sync_all();
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else
+      tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 

@@ -174,3 +174,35 @@ def make_chain_inputs(M: int | None = None, D: int | None = None, F: int | None 
         layers[name] = dict(W=W, A=A, B=B, s=s, N=n, K=k, r=r)
     dy = draw_dy(M, D, 1)
     return dict(x=x, dy=dy, layers=layers, M=M, D=D, F=F, r=r, s=s)
+
+
+def make_chain_sample(m: int, f: int, D: int | None = None, F: int | None = None, r: int | None = None,
+                      s: float | None = None, w_std: float | None = None):
+    """A bounded sample of the gated-MLP chain: its first ``m`` tokens and first ``f`` intermediate features.
+
+    Every tensor equals the matching slice of ``make_chain_inputs(D=D, F=F, ...)``: x and dY are their first m
+    rows; the gate and up W and B their first f rows; the down W and A their first f columns.  Only the
+    slices that are prefixes of a row-major stream are drawn short; the down weight and its A are drawn in
+    full and sliced.  Returned like ``make_chain_inputs`` with F = f.
+    """
+    D = CHAIN["D"] if D is None else D
+    F = CHAIN["F"] if F is None else F
+    r = CHAIN["r"] if r is None else r
+    s = CHAIN["s"] if s is None else s
+    w_std = CHAIN["w_std"] if w_std is None else w_std
+    if not (0 < f <= F and f % 64 == 0):
+        raise ValueError("f must be a positive multiple of 64 not above F")
+    x = draw_x(_streams(0), m, D)
+    layers = {}
+    for name, seed in (("gate", 2), ("up", 3)):
+        st = _streams(seed)
+        W = draw_w(st, f, D, w_std)                 # first f rows of [F, D]
+        A, _ = draw_lora(st, 0, D, r)               # A [r, D] does not depend on F
+        B = to_bf16(st[4].standard_normal((f, r), dtype=np.float32) * np.float32(0.01))  # first f rows of [F, r]
+        layers[name] = dict(W=W, A=A, B=B, s=s, N=f, K=D, r=r)
+    st = _streams(4)
+    W = np.ascontiguousarray(draw_w(st, D, F, w_std)[:, :f])
+    A, B = draw_lora(st, D, F, r)
+    layers["down"] = dict(W=W, A=A[:, :f].contiguous(), B=B, s=s, N=D, K=f, r=r)
+    dy = draw_dy(m, D, 1)
+    return dict(x=x, dy=dy, layers=layers, M=m, D=D, F=f, r=r, s=s)

@@ -27,6 +27,16 @@ _lock = threading.Lock()
 _c_i64 = ctypes.c_int64
 _c_p = ctypes.c_void_p
 
+QL_W_NF4, QL_W_NF4_DQ, QL_W_NVFP4 = 0, 1, 2
+
+
+class QlWeight(ctypes.Structure):
+    """Mirror of include/qlora.h's ql_weight."""
+    _fields_ = [("format", ctypes.c_int), ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
+                ("code8", ctypes.c_void_p), ("c1", ctypes.c_void_p), ("mu", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p)]
+
+
 # name -> (restype, argtypes): mirrors include/qlora.h
 SIGNATURES = {
     "ql_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -53,6 +63,16 @@ SIGNATURES = {
     "qlora_swiglu_bwd": (ctypes.c_int, [_c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
     "qlora_swiglu_gated_fwd": (ctypes.c_int, [_c_i64, _c_i64, _c_p, _c_p, _c_p]),
     "qlora_swiglu_gated_bwd": (ctypes.c_int, [_c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p]),
+    "qlora_linear_fwd_w": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, ctypes.POINTER(QlWeight), _c_p, _c_p,
+                                          ctypes.c_float, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
+    "qlora_linear_bwd_w": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, ctypes.POINTER(QlWeight), _c_p,
+                                          _c_p, ctypes.c_float, _c_p, _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
+    "qlora_gated_workspace_bytes": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64, _c_i64, ctypes.c_int]),
+    "qlora_gate_up_fwd_swiglu": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                                ctypes.c_float, _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
+    "qlora_down_bwd_dswiglu": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                              ctypes.c_float, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t,
+                                              _c_p]),
     "ql_formats_launch_count": (ctypes.c_uint64, []),
     "ql_formats_get_device_error": (ctypes.c_int, [_c_p]),
     "nf4_double_quantize_scratch_bytes": (ctypes.c_size_t, [_c_i64]),
@@ -260,6 +280,95 @@ def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, S: torch.Tensor,
     _check(lib().nvfp4_dequantize(_ptr(codes), _ptr(scales), _ptr(S), numel, code, _ptr(out), _stream(codes.device)),
            "nvfp4_dequantize")
     return out
+
+
+# ------------------------------------------------------------------------------------------ weights in any format
+
+
+class Weight:
+    """A frozen base weight [N, K] in one of the formats, with the device tensors it points to kept alive."""
+
+    def __init__(self, N, K, fmt, **t):
+        self.N, self.K, self.format, self.t = N, K, fmt, t
+        self.c = QlWeight(fmt, *(t[k].data_ptr() if t.get(k) is not None else None
+                                 for k in ("codes", "absmax", "code8", "c1", "mu", "scales", "tensor_scale")))
+
+    @staticmethod
+    def nf4(W):
+        codes, absmax = nf4_quantize(W.contiguous())
+        return Weight(W.shape[0], W.shape[1], QL_W_NF4, codes=codes, absmax=absmax)
+
+    @staticmethod
+    def nf4_dq(W):
+        codes, absmax = nf4_quantize(W.contiguous())
+        code8, c1, mu = nf4_double_quantize(absmax)
+        return Weight(W.shape[0], W.shape[1], QL_W_NF4_DQ, codes=codes, code8=code8, c1=c1, mu=mu)
+
+    @staticmethod
+    def nvfp4(W):
+        codes, scales, S = nvfp4_quantize(W.contiguous())
+        return Weight(W.shape[0], W.shape[1], QL_W_NVFP4, codes=codes, scales=scales, tensor_scale=S)
+
+
+def linear_fwd_w(x, w: Weight, A, B, s: float, want_su: bool = True):
+    M, K = x.shape
+    r = 0 if A is None else A.shape[0]
+    y = torch.empty(M, w.N, dtype=torch.bfloat16, device=x.device)
+    su = torch.empty(M, r, dtype=torch.bfloat16, device=x.device) if (r and want_su) else None
+    need = workspace_bytes(M, w.N, K, r, QL_PASS_FWD)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().qlora_linear_fwd_w(M, w.N, K, r, _ptr(_bits(x)), ctypes.byref(w.c), _ptr(A), _ptr(B), float(s),
+                                    _ptr(y), _ptr(su), _ptr(ws), need, _stream(x.device)), "qlora_linear_fwd_w")
+    return y, su
+
+
+def linear_bwd_w(dy, x, w: Weight, A, B, s: float, su=None):
+    M, N = dy.shape
+    K = w.K
+    r = 0 if A is None else A.shape[0]
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device=dy.device)
+    dA = torch.empty(r, K, dtype=torch.float32, device=dy.device) if r else None
+    dB = torch.empty(N, r, dtype=torch.float32, device=dy.device) if r else None
+    need = workspace_bytes(M, N, K, r, QL_PASS_BWD)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dy.device)
+    _check(lib().qlora_linear_bwd_w(M, N, K, r, _ptr(_bits(dy)), _ptr(_bits(x)), ctypes.byref(w.c), _ptr(A), _ptr(B),
+                                    float(s), _ptr(su), _ptr(dx), _ptr(dA), _ptr(dB), _ptr(ws), need,
+                                    _stream(dy.device)), "qlora_linear_bwd_w")
+    return dx, dA, dB
+
+
+# ------------------------------------------------------------------------------------------ gated MLP (fused SwiGLU)
+
+
+def gate_up_fwd_swiglu(x, layer, h):
+    """(gu [M, 2F] interleaved, h [M, F], su) for the interleaved gate/up QLoRALinear ``layer``; h is written."""
+    M, K = x.shape
+    N, r = layer.N, layer.r
+    F = N // 2
+    gu = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    su = torch.empty(M, r, dtype=torch.bfloat16, device=x.device) if r else None
+    need = int(lib().qlora_gated_workspace_bytes(M, N, K, r, QL_PASS_FWD))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().qlora_gate_up_fwd_swiglu(M, F, K, r, _ptr(_bits(x)), _ptr(layer.codes), _ptr(layer.absmax),
+                                          _ptr(layer.A if r else None), _ptr(layer.B if r else None), layer.s,
+                                          _ptr(gu), _ptr(h), _ptr(su), _ptr(ws), need, _stream(x.device)),
+           "qlora_gate_up_fwd_swiglu")
+    return gu, h, su
+
+
+def down_bwd_dswiglu(dy, h, layer, su, gu, dgu):
+    """(dgu [M, 2F] interleaved, dA, dB) for the down QLoRALinear ``layer`` (input h, output dy)."""
+    M, N = dy.shape
+    F, r = layer.K, layer.r
+    dA = torch.empty(r, F, dtype=torch.float32, device=dy.device) if r else None
+    dB = torch.empty(N, r, dtype=torch.float32, device=dy.device) if r else None
+    need = int(lib().qlora_gated_workspace_bytes(M, N, F, r, QL_PASS_BWD))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dy.device)
+    _check(lib().qlora_down_bwd_dswiglu(M, N, F, r, _ptr(_bits(dy)), _ptr(_bits(h)), _ptr(layer.codes),
+                                        _ptr(layer.absmax), _ptr(layer.A if r else None), _ptr(layer.B if r else None),
+                                        layer.s, _ptr(su), _ptr(gu), _ptr(dgu), _ptr(dA), _ptr(dB), _ptr(ws), need,
+                                        _stream(dy.device)), "qlora_down_bwd_dswiglu")
+    return dgu, dA, dB
 
 
 # ------------------------------------------------------------------------------------------ linear layer

@@ -7,9 +7,9 @@
 
 using namespace qlora;
 
-template <int BN, int AM, int KB>
+template <int BN, int AM, int KB, int EPI = EPI_PLAIN>
 void row() {
-  using C = UmmaCfg<BN, AM, false, KB>;
+  using C = UmmaCfg<BN, AM, false, KB, false, EPI>;
   std::printf("%d %d %d %d %d %d %d %d\n", BN, AM, KB, C::kQStages, C::kAStages, C::kBStages, C::kDeqGroups,
               C::kAccBufs);
 }
@@ -28,5 +28,12 @@ int main() {
   row<64, A_DEQ_MN, 1>();
   row<128, A_DEQ_MN, 1>();
   row<256, A_DEQ_MN, 1>();
+  row<16, A_DEQ_TMEM_T, 1>();
+  row<32, A_DEQ_TMEM_T, 1>();
+  row<64, A_DEQ_TMEM_T, 1>();
+  row<128, A_DEQ_TMEM_T, 1>();
+  row<256, A_DEQ_TMEM_T, 1>();
+  row<128, A_DEQ_TMEM, 1, EPI_SWIGLU_FWD>();
+  row<256, A_DEQ_TMEM, 1, EPI_SWIGLU_FWD>();
   return 0;
 }

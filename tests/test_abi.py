@@ -151,3 +151,39 @@ def test_format_conversions_reject_bad_arguments_on_host(L):
     assert lib.nvfp4_dequantize(p, p, p, 32, 9, p, None) == L.QL_ERR_INVALID_ARG
     assert lib.nvfp4_dequantize(p, p, p, 0, 0, p, None) == L.QL_ERR_INVALID_ARG
     assert L.formats_launch_count() == 0  # nothing above reached a launch
+
+
+def test_weight_descriptor_calls_reject_bad_weights_on_host(L):
+    lib = L.lib()
+    p = ctypes.c_void_p(FAKE)
+    bad = FAKE + 4
+
+    def call(w):
+        return lib.qlora_linear_fwd_w(64, 256, 256, 8, p, ctypes.byref(w) if w is not None else None, p, p, 2.0, p,
+                                      None, p, 1 << 30, None)
+    assert call(None) == L.QL_ERR_INVALID_ARG
+    assert call(L.QlWeight(7, FAKE, FAKE)) == L.QL_ERR_INVALID_ARG                       # unknown format
+    assert call(L.QlWeight(L.QL_W_NF4, FAKE, None)) == L.QL_ERR_INVALID_ARG              # absmax missing
+    assert call(L.QlWeight(L.QL_W_NF4_DQ, FAKE, None, FAKE, None, FAKE)) == L.QL_ERR_INVALID_ARG  # c1 missing
+    assert call(L.QlWeight(L.QL_W_NVFP4, FAKE, None, None, None, None, bad, FAKE)) == L.QL_ERR_INVALID_ARG
+    w = L.QlWeight(L.QL_W_NVFP4, FAKE, None, None, None, None, FAKE, FAKE)
+    assert lib.qlora_linear_bwd_w(16, 12, 64, 8, p, p, ctypes.byref(w), p, p, 2.0, None, p, p, p, p, 1 << 30,
+                                  None) == L.QL_ERR_INVALID_ARG                           # N % 8 != 0
+    assert L.formats_launch_count() == 0 and L.launch_count() == 0
+
+
+def test_gated_calls_reject_bad_arguments_on_host(L):
+    lib = L.lib()
+    p = ctypes.c_void_p(FAKE)
+    assert lib.qlora_gate_up_fwd_swiglu(64, 24, 256, 8, p, p, p, p, p, 2.0, p, p, None, p, 1 << 30, None) == \
+        L.QL_ERR_INVALID_ARG                                                               # F % 16 != 0
+    assert lib.qlora_gate_up_fwd_swiglu(64, 32, 256, 8, p, p, p, p, p, 2.0, p, None, None, p, 1 << 30, None) == \
+        L.QL_ERR_INVALID_ARG                                                               # h missing
+    assert lib.qlora_down_bwd_dswiglu(64, 256, 32, 8, p, p, p, p, p, p, 2.0, None, None, p, p, p, p, 1 << 30,
+                                      None) == L.QL_ERR_INVALID_ARG                        # gu missing
+    need = lib.qlora_gated_workspace_bytes(64, 256, 32, 8, L.QL_PASS_BWD)
+    assert lib.qlora_down_bwd_dswiglu(64, 256, 32, 8, p, p, p, p, p, p, 2.0, None, p, p, p, p, p, max(need, 1) - 1,
+                                      None) == L.QL_ERR_INVALID_ARG                        # workspace short
+    assert lib.qlora_gated_workspace_bytes(2048, 57344, 8192, 128, L.QL_PASS_FWD) == \
+        L.workspace_bytes(2048, 57344, 8192, 128, L.QL_PASS_FWD)
+    assert L.launch_count() == 0

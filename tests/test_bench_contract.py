@@ -25,7 +25,8 @@ def test_reference_arm_prints_one_contract_line():
     out = json.loads(lines[0])
     assert KEYS <= set(out)
     assert out["impl"] == "reference" and out["value"] > 0 and out["higher_is_better"] is True
-    assert out["config"]["workload"] == "attn_2048x4096x4096_r16"
+    assert out["config"]["workload"] == "mlpchain_8192x8192x28672_r64"
+    assert out["config"]["sampled_tokens_per_step"] == 16
     assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] >= 1
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["d2h_bytes_per_step"] == 0
     assert out["e2e"]["value"] == out["value"]

@@ -39,11 +39,12 @@ def test_recorded_traffic_only_for_matching_code(tmp_path, monkeypatch):
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(b, "ROOT", str(tmp_path))
     monkeypatch.setattr(b, "LAYER_SOURCES", ("k.cu",))
-    rec = {"source_sha": b.kernel_source_sha(), "kernels": {"fused_dx": 123}}
+    rec = {"source_sha": b.kernel_source_sha(), "workloads": {"wl": {"fused_dx": 123}}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
-    assert b.load_traffic() == {"fused_dx": 123}
+    assert b.load_traffic("wl") == {"fused_dx": 123}
+    assert b.load_traffic("other") == {}
     (csrc / "k.cu").write_text("int main() { return 1; }\n")
-    assert b.load_traffic() == {}
+    assert b.load_traffic("wl") == {}
 
 
 def test_hashed_sources_are_the_layer_translation_unit():
@@ -65,15 +66,33 @@ def test_hashed_sources_are_the_layer_translation_unit():
 
 
 def test_committed_traffic_record():
-    """profiles/traffic.json names both fused kernels with positive byte counts; when it was taken on the kernel
-    code in this tree the bench reports it (after a kernel change it is stale and the bench reports null)."""
+    """profiles/traffic.json names, per workload, fused kernels with positive byte counts; when it was taken on
+    the kernel code in this tree the bench reports it (after a kernel change it is stale and the bench reports
+    null)."""
     b = load_bench()
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
         rec = json.load(f)
-    assert set(rec["kernels"]) == {"fused_fwd", "fused_dx"} and all(v > 0 for v in rec["kernels"].values())
+    assert rec["workloads"] and all(v > 0 for k in rec["workloads"].values() for v in k.values())
     if rec["source_sha"] != b.kernel_source_sha():
         pytest.skip("traffic recorded before the latest kernel change: re-capture it on a B200")
-    assert b.load_traffic() == rec["kernels"]
+    for wl, kernels in rec["workloads"].items():
+        assert b.load_traffic(wl) == kernels
+
+
+def test_chain_work_counts():
+    """The block's FLOP count is the sum of its three layers' counts, and the four fused GEMMs of a step carry
+    the base products (2 M N K each) plus their LoRA products."""
+    b = load_bench()
+    from qlora_fine_tuning_blockwise_b200 import inputs as I
+    M, D, F, r = 8192, 8192, 28672, 64
+    gu = I.LinearWorkload("gu", M, D, F, r, 2.0, 0.0)
+    dn = I.LinearWorkload("dn", M, F, D, r, 2.0, 0.0)
+    ff, fb = b.chain_flops(M, D, F, r)
+    assert ff == 2 * gu.flops_fwd + dn.flops_fwd and fb == 2 * gu.flops_bwd + dn.flops_bwd
+    k = b.chain_kernel_flops(M, D, F, r)
+    assert k["gate_up_fwd"] + k["down_fwd"] == ff - 2 * (2 * M * D * r) - 2 * M * F * r  # minus the s x A^T GEMMs
+    assert k["down_dx"] == 2 * M * D * F + 2 * M * r * F and k["gate_up_dx"] == 2 * M * 2 * F * D + 4 * M * r * D
+    assert abs(ff / 1e12 - 11.66) < 0.01 and abs(fb / 1e12 - 11.78) < 0.01  # the block's 11.66 / 11.78 TFLOP
 
 
 def test_clock_summary_parses_samples_and_reasons():

@@ -1,7 +1,8 @@
 """GPU parity of the SwiGLU kernels and of the gated-MLP block (gate/up -> SwiGLU -> down) against the oracle.
 
 The oracle runs the block as three separate layers with the activations rounded to bf16 between them
-(its reading of how the block stores activations); the library fuses gate and up into one stacked layer.
+(its reading of how the block stores activations); the library fuses gate and up into one stacked layer whose
+rows interleave the two by 16, with the SwiGLU in its GEMM epilogue.
 """
 
 import numpy as np
@@ -66,6 +67,26 @@ def build_block(ops, c):
                          dev(Ls["down"]["A"]), dev(Ls["down"]["B"]), c["s"])
 
 
+def gate_up_columns(F):
+    """Columns of the stacked gate/up output that hold gate feature f and up feature f: the stacked rows are
+    interleaved by 16 (16 gate rows, then the 16 up rows of the same features)."""
+    f = torch.arange(F, device="cuda")
+    gp = (f // 16) * 32 + f % 16
+    return gp, gp + 16
+
+
+def check_grads(grads, rgrads, F):
+    """dA, dB of each layer against the oracle; the gate and up dB come as [F / 16, 16, r] views of the stacked
+    gradient (feature 16 q + i at [q, i])."""
+    for name in ("gate", "up", "down"):
+        dA, dB = grads[name]
+        if name != "down":
+            assert dB.shape[:2] == (F // 16, 16)
+            dB = dB.reshape(F, -1)
+        assert_close(dA, rgrads[name][0], f"dA {name}")
+        assert_close(dB, rgrads[name][1], f"dB {name}")
+
+
 def oracle_layers(c):
     out = {}
     for name, Ld in c["layers"].items():
@@ -85,14 +106,13 @@ def test_gated_mlp_block_small(ops, M, D, F, r):
     Lo = oracle_layers(c)
     ry, g, u, h = L.mlp_chain_forward(f64(c["x"]), Lo["gate"], Lo["up"], Lo["down"])
     rdx, rgrads = L.mlp_chain_backward(f64(c["dy"]), f64(c["x"]), Lo["gate"], Lo["up"], Lo["down"], (g, u, h))
-    assert_close(saved[0][:, :F], g, "g")
-    assert_close(saved[0][:, F:], u, "up")
+    gp, up = gate_up_columns(F)
+    assert_close(saved[0][:, gp], g, "g")
+    assert_close(saved[0][:, up], u, "up")
     assert_close(saved[2], h, "h")
     assert_close(y, ry, "y")
     assert_close(dx, rdx, "dX")
-    for name in ("gate", "up", "down"):
-        assert_close(grads[name][0], rgrads[name][0], f"dA {name}")
-        assert_close(grads[name][1], rgrads[name][1], f"dB {name}")
+    check_grads(grads, rgrads, F)
 
 
 def test_gated_mlp_block_full_size_sampled(ops):
@@ -122,6 +142,4 @@ def test_gated_mlp_block_full_size_sampled(ops):
     torch.cuda.synchronize()
     ry, g, u, h = L.mlp_chain_forward(f64(c["x"])[:Ms], Lo["gate"], Lo["up"], Lo["down"])
     _, rgrads = L.mlp_chain_backward(f64(c["dy"])[:Ms], f64(c["x"])[:Ms], Lo["gate"], Lo["up"], Lo["down"], (g, u, h))
-    for name in ("gate", "up", "down"):
-        assert_close(grads[name][0], rgrads[name][0], f"dA {name}")
-        assert_close(grads[name][1], rgrads[name][1], f"dB {name}")
+    check_grads(grads, rgrads, c["F"])

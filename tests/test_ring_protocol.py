@@ -288,7 +288,7 @@ def kernel_depths(tmpdir):
 def test_every_instantiation_is_safe_under_random_schedules(tmp_path):
     """The model with the depths each dequantizing kernel instantiation actually uses (not a copy of them)."""
     rows = kernel_depths(str(tmp_path))
-    assert len(rows) == 13
+    assert len(rows) == 20
     for BN, AM, KB, QS, AS, BS, G, acc in sorted({r for r in rows}):
         assert QS >= AS + G and G <= AS, (BN, AM, KB)
         cfg = Cfg(QS, AS, BS, G, UNITS, acc_bufs=acc)

@@ -58,9 +58,11 @@ def load_peaks() -> dict:
 
 
 # The sources of the layer library (libqlora's qlora.cu translation unit and what it includes): the kernels
-# whose counters are recorded under profiles/ are built from these and nothing else.  The format conversions
-# (formats.cu, formats.cuh) are a separate translation unit that none of them includes.
-LAYER_SOURCES = ("elementwise.cuh", "nf4_table.cuh", "ptx.cuh", "qlora.cu", "swiglu.cuh", "umma_gemm.cuh")
+# whose counters are recorded under profiles/ are built from these and nothing else.  The format conversions'
+# kernels (formats.cu) are a separate translation unit; their per-element arithmetic (formats.cuh) is shared
+# with the FP4 path's activation quantizer.
+LAYER_SOURCES = ("elementwise.cuh", "formats.cuh", "fp4_gemm.cuh", "nf4_table.cuh", "ptx.cuh", "qlora.cu",
+                 "swiglu.cuh", "umma_gemm.cuh")
 
 
 def kernel_source_sha() -> str:

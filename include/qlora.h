@@ -370,6 +370,46 @@ QL_API ql_status nvfp4_quantize(const float* w, int64_t numel, uint8_t* codes, u
 QL_API ql_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
                                   int64_t numel, ql_dtype out_dtype, void* out, void* stream);
 
+/*
+ * The NVFP4 form of the layer on the block-scaled FP4 tensor core ("Major Unsloth Update: NVFP4 Quantization Export
+ * and DeepSeek-V4 Training Support" (kongchang.com), section "NVFP4: A Quantization Format for the Next Generation
+ * of Hardware": E2M1 values sharing an FP8 scale per group, multiplied directly by Blackwell's FP4 tensor cores).
+ *
+ * nvfp4_scales_to_mma -- lays a weight's NVFP4 scales (nvfp4_quantize's row-major [rows, K/16] E4M3 bytes) out as
+ * the tensor core reads them: rows in blocks of 128, K in steps of 64 elements (4 scales), one 512-byte atom per
+ * (row block, step), the steps of a row block consecutive and padded with zero scales to a multiple of 4, row
+ * blocks consecutive; inside an atom the scale of group g of row 32 r1 + r0 is byte 16 r0 + 4 r1 + g.  Rows past
+ * `rows` up to the next multiple of 128 hold zero scales.
+ *   rows >= 1, K >= 64 with K % 64 == 0; out 16-byte aligned, nvfp4_mma_scales_bytes(rows, K) bytes.  Runs once
+ *   per frozen weight.
+ */
+QL_API size_t nvfp4_mma_scales_bytes(int64_t rows, int64_t K);
+QL_API ql_status nvfp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* out, void* stream);
+
+/*
+ * qlora_linear_fwd_fp4 -- y = q(x) q(W)^T + s (x A^T) B^T, with q() the NVFP4 rule of nvfp4_quantize (E2M1 codes,
+ * an E4M3 scale per 16 elements along K, one fp32 tensor scale per operand).  The weight comes quantized (codes,
+ * its scales in the MMA layout of nvfp4_scales_to_mma, its tensor scale on the device); the activations are
+ * quantized by the same rule on every call, with their own tensor scale, into the workspace.  The base product
+ * runs as tcgen05.mma kind::mxf4nvf4 with 16-element scale blocks into one TMEM accumulator, scaled by both tensor
+ * scales in the epilogue; the rank-r term keeps the unquantized activations: su = s x A^T is rounded to bf16 and
+ * multiplied by B with bf16 MMAs into a second accumulator.
+ *   M, N, K, r   as qlora_linear_fwd (K % 64 == 0, N % 8 == 0, r % 8 == 0, r <= 256).
+ *   x            bf16 [M,K], 16-byte aligned.
+ *   w_codes      uint8 [N, K/2]: E2M1 codes, element 2j in the low nibble of byte j (nvfp4_quantize of W [N,K]).
+ *   w_sf_mma     the weight's scales in the MMA layout, w_S its fp32 tensor scale (device).
+ *   A, B, s      the LoRA pair and scaling (unused when r = 0).
+ *   y            bf16 [M,N] out; su_out nullable bf16 [M,r] out (s x A^T).
+ *   workspace    qlora_fp4_workspace_bytes(M,N,K,r) bytes: the activations' codes, scales and tensor scale, su.
+ * Errors as qlora_linear_fwd; a non-finite activation sets the device error word (QL_ERR_INVALID_ARG from
+ * ql_get_device_error).
+ */
+QL_API size_t qlora_fp4_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r);
+QL_API ql_status qlora_linear_fwd_fp4(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x,
+                                      const uint8_t* w_codes, const uint8_t* w_sf_mma, const float* w_S,
+                                      const uint16_t* A, const uint16_t* B, float s, uint16_t* y, uint16_t* su_out,
+                                      void* workspace, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

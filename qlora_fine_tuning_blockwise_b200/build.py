@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqlora.so")
 SOURCES = [os.path.join(CSRC, "qlora.cu"), os.path.join(CSRC, "formats.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "umma_gemm.cuh", "elementwise.cuh", "nf4_table.cuh", "formats.cuh", "swiglu.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "umma_gemm.cuh", "elementwise.cuh", "nf4_table.cuh", "formats.cuh", "swiglu.cuh", "fp4_gemm.cuh")] + [
     os.path.join(ROOT, "include", "qlora.h")
 ]
 

@@ -356,6 +356,35 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
+// ------------------------------------------------------------------------------------------ block-scaled FP4
+
+// Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both addresses 16-byte aligned), completing as
+// transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Shared -> tensor memory copy of 32 rows x 16 bytes (the source: rows 16 bytes apart, described by `sdesc`),
+// row i to lane i and to lanes i + 32, i + 64, i + 96 (one copy per TMEM lane quarter), 16 bytes = 4 consecutive
+// 32-bit columns from `taddr`.  Asynchronous; ordered before the tcgen05.mma the same thread issues after it.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// D[tmem] (+)= (A . SFA) * (B . SFB)^T with A, B packed E2M1 (K-major, 64 elements = 32 bytes per row per
+// instruction) and one UE4M3 scale per 16 elements of a row, read from tensor memory at sfa / sfb; fp32 D.
+__device__ __forceinline__ void umma_fp4_block16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // ------------------------------------------------------------------------------------------ descriptors
 
 // Shared-memory matrix descriptor, SWIZZLE_128B canonical layouts (sm_100 "version 1" descriptor).
@@ -371,6 +400,26 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
   d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
   return d;
+}
+
+// Shared-memory matrix descriptor, no swizzle, K-major: core matrices of 8 rows x 16 bytes (rows 16 bytes apart),
+// successive 8-row core matrices `sbo` bytes apart.  Used for the tcgen05.cp source of scale factors.
+__device__ __forceinline__ uint64_t sdesc_noswizzle(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
+  return d;                             // layout type 0: no swizzle
+}
+
+// Instruction descriptor for kind::mxf4nvf4 with 16-element scale blocks: E2M1 A and B (format code 1), UE4M3
+// scale factors (scale-format bit 0), both K-major, fp32 D, M x N tile, K = 64 per instruction, scale-factor
+// byte ids 0 (all four bytes of a TMEM word serve one 64-element step).
+__host__ __device__ constexpr uint32_t idesc_fp4_block16(int M, int N) {
+  return (1u << 7)                                   // A format: E2M1
+         | (1u << 10)                                // B format: E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
 // Instruction descriptor for kind::f16: bf16 A and B, fp32 D, M x N tile, operand majorness.

@@ -12,6 +12,7 @@
 
 #include "../../include/qlora.h"
 #include "elementwise.cuh"
+#include "fp4_gemm.cuh"
 #include "umma_gemm.cuh"
 
 namespace qlora {
@@ -1139,6 +1140,162 @@ ql_status qlora_swiglu_gated_bwd(int64_t M, int64_t F, const uint16_t* dh, const
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------ NVFP4 forward
+
+namespace qlora {
+namespace {
+
+// Workspace of qlora_linear_fwd_fp4: [x codes M x K/2][x scales, MMA layout][x tensor scale][su bf16 M x r]
+// [fp32 partials of the split s x A^T product].
+struct Fp4Plan {
+  size_t off_codes = 0, off_sf = 0, off_S = 0, off_su = 0, off_part = 0, total = 0;
+  int s_su = 1;
+};
+
+Fp4Plan plan_fp4(int64_t M, int64_t N, int64_t K, int64_t r) {
+  Fp4Plan p;
+  const LinearPlan lp = plan_linear(M, N, K, r, QL_PASS_FWD);
+  size_t off = 0;
+  p.off_codes = off;
+  off += align256(static_cast<size_t>(M) * K / 2);
+  p.off_sf = off;
+  off += align256(static_cast<size_t>(fp4_sf_bytes(M, K)));
+  p.off_S = off;
+  off += 256;
+  if (r > 0) {
+    p.off_su = off;
+    off += align256(static_cast<size_t>(M) * r * 2);
+    p.s_su = lp.s_su;
+    p.off_part = off;
+    if (lp.s_su > 1) off += align256(static_cast<size_t>(lp.s_su) * M * r * 4);
+  }
+  p.total = off;
+  return p;
+}
+
+cudaError_t launch_fp4_gemm(int64_t M, int64_t N, int64_t K, int64_t r, const uint8_t* w_codes, const uint8_t* w_sf,
+                            const float* w_S, const uint8_t* x_codes, const uint8_t* x_sf, const float* x_S,
+                            const uint16_t* B, const uint16_t* su, uint16_t* y, unsigned int* err, int sms,
+                            cudaStream_t stream) {
+  constexpr int BN = 128;
+  using C = Fp4Cfg<BN>;
+  CUtensorMap tmA, tmB, tmLA, tmLB;
+  std::memset(&tmLA, 0, sizeof(tmLA));
+  std::memset(&tmLB, 0, sizeof(tmLB));
+  if (!make_map(&tmA, w_codes, N, K / 2, 1, 128, 128, true)) return cudaErrorInvalidValue;
+  if (!make_map(&tmB, x_codes, M, K / 2, 1, 128, BN, true)) return cudaErrorInvalidValue;
+  if (r > 0) {
+    if (!make_map(&tmLA, B, N, r, 2, 64, 128, true)) return cudaErrorInvalidValue;
+    if (!make_map(&tmLB, su, M, r, 2, 64, BN, true)) return cudaErrorInvalidValue;
+  }
+  Fp4Args a{};
+  a.rows = static_cast<int>(N);
+  a.cols = static_cast<int>(M);
+  a.tiles_i = static_cast<int>(cdiv(N, 128));
+  a.tiles_j = static_cast<int>(cdiv(M, BN));
+  a.k_stages = static_cast<int>(cdiv(K, 256));
+  a.n_extra = r > 0 ? static_cast<int>(cdiv(r, 64)) : 0;
+  a.sfa = w_sf;
+  a.sfb = x_sf;
+  a.sf_rb_bytes = fp4_sf_rowblock_bytes(K);
+  a.Sa = w_S;
+  a.Sb = x_S;
+  a.out = reinterpret_cast<__nv_bfloat16*>(y);
+  a.ld = N;
+  a.rows_lim = static_cast<int>(N);
+  a.cols_lim = static_cast<int>(M);
+  a.err = err;
+  const int64_t units = static_cast<int64_t>(a.tiles_i) * a.tiles_j;
+  // both operands are 0.5625 bytes per element, so the balanced group is about sqrt(C) weight tiles (see
+  // unit_group)
+  a.group_i = 0;
+  if (grouped_enabled() && a.tiles_j > 1 && units > sms) {
+    int gi = static_cast<int>(std::lround(std::sqrt(static_cast<double>(sms) * BN / 128.0)));
+    a.group_i = std::max(1, std::min(gi, a.tiles_i));
+  }
+  auto kern = fp4_gemm_kernel<BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, sms)));
+  prof_record(0, 0, stream);
+  kern<<<grid, 192, C::kSmemBytes, stream>>>(tmA, tmB, tmLA, tmLB, a);
+  count_launch();
+  prof_record(0, 1, stream);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace qlora
+
+extern "C" size_t nvfp4_mma_scales_bytes(int64_t rows, int64_t K) {
+  if (rows < 1 || K < 64 || K % 64 != 0) return 0;
+  return static_cast<size_t>(fp4_sf_bytes(rows, K));
+}
+
+extern "C" ql_status nvfp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* out, void* stream) {
+  if (rows < 1 || K < 64 || K % 64 != 0 || !scales || !out || !aligned16(out)) return QL_ERR_INVALID_ARG;
+  if (rows > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1) return QL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (!device_info(&d)) return QL_ERR_CUDA;
+  cudaStream_t cs = as_stream(stream);
+  if (cudaMemsetAsync(out, 0, static_cast<size_t>(fp4_sf_bytes(rows, K)), cs) != cudaSuccess) return QL_ERR_CUDA;
+  const long long n = rows * (K / 16);
+  fp4_sf_to_mma_kernel<<<static_cast<unsigned>(std::min<long long>(cdiv(n, 256), d.sms * 16LL)), 256, 0, cs>>>(
+      scales, rows, K, out);
+  count_launch();
+  return status_of(cudaGetLastError());
+}
+
+extern "C" size_t qlora_fp4_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r) {
+  if (check_linear(M, N, K, r) != QL_OK || M == 0) return 0;
+  return plan_fp4(M, N, K, r).total;
+}
+
+extern "C" ql_status qlora_linear_fwd_fp4(int64_t M, int64_t N, int64_t K, int64_t r, const uint16_t* x,
+                                          const uint8_t* w_codes, const uint8_t* w_sf_mma, const float* w_S,
+                                          const uint16_t* A, const uint16_t* B, float s, uint16_t* y,
+                                          uint16_t* su_out, void* workspace, size_t ws_bytes, void* stream) {
+  ql_status st = check_linear(M, N, K, r);
+  if (st != QL_OK) return st;
+  if (M == 0) return QL_OK;
+  if (!x || !w_codes || !w_sf_mma || !w_S || !y || !aligned16(x) || !aligned16(w_codes) || !aligned16(w_sf_mma) ||
+      !aligned16(y))
+    return QL_ERR_INVALID_ARG;
+  if (r > 0 && (!A || !B || !aligned16(A) || !aligned16(B))) return QL_ERR_INVALID_ARG;
+  if (su_out && !aligned16(su_out)) return QL_ERR_INVALID_ARG;
+  const Fp4Plan p = plan_fp4(M, N, K, r);
+  if (ws_bytes < p.total || !workspace || !aligned16(workspace)) return QL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (!device_info(&d)) return QL_ERR_CUDA;
+  cudaStream_t cs = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* x_codes = ws + p.off_codes;
+  uint8_t* x_sf = ws + p.off_sf;
+  float* x_S = reinterpret_cast<float*>(ws + p.off_S);
+  // the activations in NVFP4: largest magnitude, blocks (scales straight into the MMA layout), tensor scale
+  if (cudaMemsetAsync(x_sf, 0, static_cast<size_t>(fp4_sf_bytes(M, K)), cs) != cudaSuccess) return QL_ERR_CUDA;
+  if (cudaMemsetAsync(x_S, 0, sizeof(float), cs) != cudaSuccess) return QL_ERR_CUDA;
+  const long long numel = M * K, nblk = numel / 16;
+  const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  fp4_act_amax_kernel<<<static_cast<unsigned>(std::min<long long>(cdiv(numel, 256 * 8), d.sms * 16LL)), 256, 0, cs>>>(
+      xb, numel, reinterpret_cast<unsigned int*>(x_S), d.err);
+  count_launch();
+  fp4_act_quantize_kernel<<<static_cast<unsigned>(std::min<long long>(cdiv(nblk, 256), d.sms * 16LL)), 256, 0, cs>>>(
+      xb, M, K, reinterpret_cast<const unsigned int*>(x_S), x_codes, x_sf);
+  count_launch();
+  fp4_act_finalize_kernel<<<1, 32, 0, cs>>>(x_S);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return QL_ERR_CUDA;
+  uint16_t* su = nullptr;
+  if (r > 0) {
+    su = su_out ? su_out : reinterpret_cast<uint16_t*>(ws + p.off_su);
+    float* part = reinterpret_cast<float*>(ws + p.off_part);
+    if (run_su(M, K, r, x, A, s, su, p.s_su, part, d.err, cs) != cudaSuccess) return QL_ERR_CUDA;
+  }
+  return status_of(launch_fp4_gemm(M, N, K, r, w_codes, w_sf_mma, w_S, x_codes, x_sf, x_S, B, su, y, d.err, d.sms,
+                                   cs));
+}
 
 // ------------------------------------------------------------------------------------------ no-allocation forward
 //

@@ -80,6 +80,11 @@ SIGNATURES = {
     "nf4_double_dequantize": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i64, _c_p, _c_p]),
     "nvfp4_quantize": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_p, _c_p, _c_p]),
     "nvfp4_dequantize": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i64, ctypes.c_int, _c_p, _c_p]),
+    "nvfp4_mma_scales_bytes": (ctypes.c_size_t, [_c_i64, _c_i64]),
+    "nvfp4_scales_to_mma": (ctypes.c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p]),
+    "qlora_fp4_workspace_bytes": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64, _c_i64]),
+    "qlora_linear_fwd_fp4": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                            ctypes.c_float, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p]),
 }
 
 
@@ -369,6 +374,57 @@ def down_bwd_dswiglu(dy, h, layer, su, gu, dgu):
                                         layer.s, _ptr(su), _ptr(gu), _ptr(dgu), _ptr(dA), _ptr(dB), _ptr(ws), need,
                                         _stream(dy.device)), "qlora_down_bwd_dswiglu")
     return dgu, dA, dB
+
+
+def nvfp4_scales_to_mma(scales: torch.Tensor, rows: int, K: int) -> torch.Tensor:
+    """An NVFP4 weight's row-major scales [rows, K/16] laid out as the FP4 tensor core reads them (uint8)."""
+    assert scales.is_cuda and scales.dtype == torch.uint8
+    out = torch.empty(int(lib().nvfp4_mma_scales_bytes(rows, K)), dtype=torch.uint8, device=scales.device)
+    _check(lib().nvfp4_scales_to_mma(_ptr(scales), rows, K, _ptr(out), _stream(scales.device)), "nvfp4_scales_to_mma")
+    return out
+
+
+class FP4Linear:
+    """A frozen base weight in NVFP4 with its bf16 LoRA pair, for the forward on the block-scaled FP4 tensor core
+    (qlora_linear_fwd_fp4): the weight is quantized once and its scales laid out for the MMA."""
+
+    def __init__(self, W: torch.Tensor, A, B, s: float):
+        assert W.dim() == 2 and W.is_cuda
+        self.N, self.K = W.shape
+        self.codes, scales, self.S = nvfp4_quantize(W.contiguous())
+        self.sf = nvfp4_scales_to_mma(scales, self.N, self.K)
+        self.A, self.B, self.s = A, B, float(s)
+        self.r = 0 if A is None else A.shape[0]
+        self._ws = {}
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, su: torch.Tensor | None = None,
+                want_su: bool = False):
+        M = x.shape[0]
+        N, K, r = self.N, self.K, self.r
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
+        if want_su and r and su is None:
+            su = torch.empty(M, r, dtype=torch.bfloat16, device=x.device)
+        ws = self._ws.get(M)
+        if ws is None:
+            ws = self._ws[M] = torch.empty(max(int(lib().qlora_fp4_workspace_bytes(M, N, K, r)), 16),
+                                           dtype=torch.uint8, device=x.device)
+        _check(lib().qlora_linear_fwd_fp4(M, N, K, r, _ptr(_bits(x)), _ptr(self.codes), _ptr(self.sf), _ptr(self.S),
+                                          _ptr(self.A if r else None), _ptr(self.B if r else None), self.s, _ptr(y),
+                                          _ptr(su), _ptr(ws), ws.numel(), _stream(x.device)), "qlora_linear_fwd_fp4")
+        return y, su
+
+    def quantized_activations(self, M: int):
+        """(codes [M, K/2], scales in the MMA layout, tensor scale) of the last forward's activations, views of the
+        workspace (the layout of qlora_linear_fwd_fp4's workspace: codes, then scales, then the tensor scale)."""
+        ws = self._ws[M]
+        K = self.K
+        ncodes = M * K // 2
+        a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+        nsf = int(lib().nvfp4_mma_scales_bytes(M, K))
+        codes = ws[:ncodes]
+        sf = ws[a256(ncodes):a256(ncodes) + nsf]
+        S = ws[a256(ncodes) + a256(nsf):a256(ncodes) + a256(nsf) + 4].view(torch.float32)
+        return codes, sf, S
 
 
 # ------------------------------------------------------------------------------------------ linear layer

@@ -752,6 +752,31 @@ def run_other_workloads(peaks, dev):
             torch.cuda.empty_cache()
         except Exception as e:  # pragma: no cover - reported, never fatal for the main line
             res[name] = {"error": f"{type(e).__name__}: {e}"[:200]}
+    # The NVFP4 form of the layer on the block-scaled FP4 tensor core: the layer forward (activation quantization,
+    # s x A^T, the FP4 GEMM) and the FP4 GEMM alone.  Its peak is the measured bf16 peak times 4, the ratio of
+    # the nominal dense FP4 and bf16 tensor rates (9 and 2.25 PFLOP/s).
+    fp4_peak = 4.0 * peaks["bf16_tflops"]
+    for name in ("attn_2048x4096x4096_r16", "mlpdown_4096x11008x4096_r64", "decode_16x8192x28672_r16"):
+        try:
+            w = I.WORKLOADS[name]
+            d = I.make_linear_inputs(w)
+            layer = ops.FP4Linear(torch.from_numpy(d["W"]).to(dev), d["A"].to(dev), d["B"].to(dev), d["s"])
+            x = d["x"].to(dev)
+            M, N, K, r = w.M, w.N, w.K, w.r
+            f_ms = timeit(lambda: layer.forward(x))
+            k_ms = kernel_ms(lambda: layer.forward(x), 0)
+            kfl = 2 * M * N * K + 2 * M * N * r
+            wbytes = N * K // 2 + N * K // 16 + 2 * M * K + 2 * M * N  # fp4 weight + its scales, x in, y out
+            res["fp4_" + name] = {
+                "fwd_ms": round(f_ms, 4), "fwd_tflops": round(w.flops_fwd / (f_ms * 1e-3) / 1e12, 1),
+                "fp4_gemm_ms": round(k_ms, 4), "fp4_gemm_tflops": round(kfl / (k_ms * 1e-3) / 1e12, 1),
+                "fp4_gemm_frac_of_fp4_peak": round(kfl / (k_ms * 1e-3) / 1e12 / fp4_peak, 4),
+                "fp4_gemm_gbs": round(wbytes / (k_ms * 1e-3) / 1e9, 1),
+                "fp4_peak_tflops": fp4_peak, "peak_note": "4 x measured bf16 (nominal dense FP4 / bf16 ratio)"}
+            del layer, x, d
+            torch.cuda.empty_cache()
+        except Exception as e:  # pragma: no cover - reported, never fatal for the main line
+            res["fp4_" + name] = {"error": f"{type(e).__name__}: {e}"[:200]}
     # NF4 round trip on the attention-projection weight (4096 x 4096)
     w = I.WORKLOADS["attn_2048x4096x4096_r16"]
     W = torch.from_numpy(I.draw_w(I._streams(0), w.N, w.K, w.w_std)).to(dev).reshape(-1)

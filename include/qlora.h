@@ -83,6 +83,18 @@ QL_API ql_status ql_set_profile_events(int which, void* start, void* stop);
 QL_API ql_status ql_selftest_wait_timeout(int64_t wait_cycles, void* stream);
 
 /*
+ * ql_selftest_arm_gemm_stall -- failure-path test hook (the paper has no counterpart).  Arms the NEXT dequantizing
+ * GEMM launch of this process (the fused forward or dX kernel of any layer call) so that one warp role leaves
+ * before doing anything: role 1 the MMA issuer, 2 the activation (B) producer, 3 the codes producer.  None of them
+ * then has a copy or an MMA in flight.  Every wait of that launch is bounded by wait_cycles (>= 100000) instead
+ * of about 2 s, so the other roles' waits expire: the kernel raises its abort flag, drains the copies it issued,
+ * frees its tensor memory and returns; ql_get_device_error then reports QL_ERR_TIMEOUT and the call's outputs
+ * are undefined.  Role 3 with r > 0 lets the LoRA stages reach the MMA before the stall, so use it with r = 0.
+ * The arming is consumed by that one launch.
+ */
+QL_API ql_status ql_selftest_arm_gemm_stall(int role, int64_t wait_cycles);
+
+/*
  * nf4_quantize -- blockwise NF4 quantization of a frozen base weight ("How LoRA and QLoRA work", as above).
  *   w        [numel] fp32, the flat row-major weight (W [N,K] gives numel = N*K).
  *   numel    number of elements; a positive multiple of `blocksize`.

@@ -81,14 +81,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 #define QLORA_IDLE_SLEEP_NS 64
 #endif
 __device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                               unsigned int* err) {
+                                               unsigned int* err, long long limit = kWaitTimeoutCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     __nanosleep(QLORA_IDLE_SLEEP_NS);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitTimeoutCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       atomicOr(err, kDevErrTimeout);
       return false;
@@ -287,7 +287,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 
 // Bounded wait with acquire at cluster scope (for barriers the peer CTA also arrives on).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                                  unsigned int* err) {
+                                                  unsigned int* err, long long limit = kWaitTimeoutCycles) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
@@ -295,7 +295,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitTimeoutCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       atomicOr(err, kDevErrTimeout);
       return false;

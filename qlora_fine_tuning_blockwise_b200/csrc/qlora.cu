@@ -362,7 +362,26 @@ cudaError_t launch_epi(const GemmCall& g, cudaStream_t stream) {
   }
 }
 
+// One-shot failure-path test (ql_selftest_arm_gemm_stall): the next dequantizing GEMM launch carries it.
+std::atomic<int> g_test_stall{0};
+std::atomic<long long> g_test_wait{0};
+
+cudaError_t launch_gemm_impl(const GemmCall& g, cudaStream_t stream);
+
 cudaError_t launch_gemm(const GemmCall& g, cudaStream_t stream) {
+  if ((g.am == A_DEQ_TMEM || g.am == A_DEQ_MN || g.am == A_DEQ_TMEM_T) && g_test_stall.load() != 0) {
+    const int role = g_test_stall.exchange(0);
+    if (role != 0) {
+      GemmCall t = g;
+      t.args.test_stall = role;
+      t.args.wait_limit = g_test_wait.load();
+      return launch_gemm_impl(t, stream);
+    }
+  }
+  return launch_gemm_impl(g, stream);
+}
+
+cudaError_t launch_gemm_impl(const GemmCall& g, cudaStream_t stream) {
   if (g.args.epi != EPI_PLAIN) {
     if (g.args.splits != 1 || g.kb != 1 || g.b_mn || g.pair || g.args.wfmt != WF_NF4) return cudaErrorInvalidValue;
     if (g.args.epi == EPI_SWIGLU_FWD && g.am == A_DEQ_TMEM) return launch_epi<A_DEQ_TMEM, EPI_SWIGLU_FWD>(g, stream);
@@ -893,6 +912,13 @@ ql_status ql_set_profile_events(int which, void* start, void* stop) {
   if (which < 0 || which > 1) return QL_ERR_INVALID_ARG;
   g_prof_events[which][0].store(start);
   g_prof_events[which][1].store(stop);
+  return QL_OK;
+}
+
+ql_status ql_selftest_arm_gemm_stall(int role, int64_t wait_cycles) {
+  if (role < 1 || role > 3 || wait_cycles < 100000 || wait_cycles > (int64_t(1) << 32)) return QL_ERR_INVALID_ARG;
+  g_test_wait.store(wait_cycles);
+  g_test_stall.store(role);
   return QL_OK;
 }
 

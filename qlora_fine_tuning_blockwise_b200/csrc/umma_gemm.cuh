@@ -118,6 +118,11 @@ struct UmmaArgs {
   // cluster split-K (TMA modes): cred = S > 1 runs the S splits of one tile as the S CTAs of a cluster, which
   // sum their fp32 partial tiles through distributed shared memory instead of writing slabs (0: off)
   int cred;
+  // failure-path test only (0 in every real launch): test_stall = 1, 2 or 3 makes the MMA issuer, the B producer
+  // or the codes producer leave before doing anything -- none of them then has a copy or an MMA in flight -- so
+  // that every other role's wait expires; wait_limit (cycles, > 0) replaces the ~2 s bound of every wait
+  int test_stall;
+  long long wait_limit;
   // unit order: group_i > 0 walks the tiles in groups of group_i tile rows (weight tiles), tile rows fastest
   // within a group, so that one wave of CTAs shares a few activation tiles and a group of weight tiles and
   // both stay in L2; 0 keeps tile columns fastest
@@ -324,6 +329,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_units = args.splits * args.tiles_i * args.tiles_j;
+  const long long lim = args.wait_limit > 0 ? args.wait_limit : kWaitTimeoutCycles;
   // CTA pairs: the even CTA of the cluster (rank 0) is the leader -- it issues the pair's MMAs, and its barriers
   // gather both CTAs' arrivals; each pair walks the units together
   const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
@@ -390,13 +396,13 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
     // ------------------------------------------------------------------ B producer
     Armed armed;
     int g = 0;
-    bool stop = false;
+    bool stop = args.test_stall == 2;
     for (int u = first_unit; u < num_units && !stop; u += unit_step) {
       const Unit U = unit_of(args, u, BN, C::kPair, rank);
       for (int it = 0; it < U.n_total; ++it, ++g) {
         const int s = g % BS;
         const uint32_t ph = static_cast<uint32_t>(g / BS) & 1u;
-        const bool ok = mbar_wait_idle(&b_empty[s], ph ^ 1u, abort_flag, args.err);
+        const bool ok = mbar_wait_idle(&b_empty[s], ph ^ 1u, abort_flag, args.err, lim);
         if (!__all_sync(kFull, ok)) {
           stop = true;
           break;
@@ -450,12 +456,12 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
     // barriers the peer CTA also arrives on are waited with acquire at cluster scope
     auto wait_mma = [&](uint64_t* bar, uint32_t par) {
       if constexpr (PAIR)
-        return mbar_wait_cluster(bar, par, abort_flag, args.err);
+        return mbar_wait_cluster(bar, par, abort_flag, args.err, lim);
       else
-        return mbar_wait(bar, par, abort_flag, args.err);
+        return mbar_wait(bar, par, abort_flag, args.err, lim);
     };
     int g = 0, lu = 0;
-    bool stop = rank != 0;  // the pair's follower issues nothing
+    bool stop = rank != 0 || args.test_stall == 1;  // the pair's follower issues nothing
     for (int u = first_unit; u < num_units && !stop; u += unit_step, ++lu) {
       const Unit U = unit_of(args, u, BN, C::kPair, rank);
       const int acc = lu % C::kAccBufs;
@@ -472,7 +478,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
           ok = wait_mma(&a_full[as], static_cast<uint32_t>(g / AS) & 1u) &&
                wait_mma(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u);
         } else {
-          ok = mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err);
+          ok = mbar_wait(&b_full[bs], static_cast<uint32_t>(g / BS) & 1u, abort_flag, args.err, lim);
         }
         if (!__all_sync(kFull, ok)) {
           stop = true;
@@ -532,7 +538,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
     for (int u = first_unit; u < num_units; u += unit_step, ++lu) {
       const Unit U = unit_of(args, u, BN, C::kPair, rank);
       const int acc = lu % C::kAccBufs;
-      int ok = mbar_wait_idle(&tmem_full[acc], static_cast<uint32_t>(lu / C::kAccBufs) & 1u, abort_flag, args.err) ? 1 : 0;
+      int ok = mbar_wait_idle(&tmem_full[acc], static_cast<uint32_t>(lu / C::kAccBufs) & 1u, abort_flag, args.err, lim) ? 1 : 0;
       tc_fence_after();
       ok = __shfl_sync(kFull, ok && !*abort_flag, 0);
       if (!ok) break;
@@ -653,13 +659,13 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
     if constexpr (C::kDeq) {
       Armed armed;
       int q = 0;
-      bool stop = false;
+      bool stop = args.test_stall == 3;
       for (int u = first_unit; u < num_units && !stop; u += unit_step) {
         const Unit U = unit_of(args, u, BN, C::kPair, rank);
         for (int it = U.n_extra; it < U.n_total; ++it, ++q) {
           const int s = q % QS;
           const uint32_t ph = static_cast<uint32_t>(q / QS) & 1u;
-          const bool ok = mbar_wait_idle(&q_empty[s], ph ^ 1u, abort_flag, args.err);
+          const bool ok = mbar_wait_idle(&q_empty[s], ph ^ 1u, abort_flag, args.err, lim);
           if (!__all_sync(kFull, ok)) {
             stop = true;
             break;
@@ -749,7 +755,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
           uint32_t r[32];  // the stage's 64 bf16 values (the first block's), packed in pairs
           if (!extra) {
             const int qs = qi % QS;
-            const bool okq = mbar_wait_idle(&q_full[qs], static_cast<uint32_t>(qi / QS) & 1u, abort_flag, args.err);
+            const bool okq = mbar_wait_idle(&q_full[qs], static_cast<uint32_t>(qi / QS) & 1u, abort_flag, args.err, lim);
             if (!__all_sync(kFull, okq)) {
               stop = true;
               break;
@@ -900,7 +906,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
           }
           // the A slot is free once the MMAs of its previous stage have completed
           const int as = g % AS;
-          const bool oka = mbar_wait_idle(&a_empty[as], (static_cast<uint32_t>(g / AS) & 1u) ^ 1u, abort_flag, args.err);
+          const bool oka = mbar_wait_idle(&a_empty[as], (static_cast<uint32_t>(g / AS) & 1u) ^ 1u, abort_flag, args.err, lim);
           if (!__all_sync(kFull, oka)) {
             stop = true;
             break;

@@ -46,6 +46,7 @@ SIGNATURES = {
     "ql_launch_count": (ctypes.c_uint64, []),
     "ql_set_profile_events": (ctypes.c_int, [ctypes.c_int, _c_p, _c_p]),
     "ql_selftest_wait_timeout": (ctypes.c_int, [_c_i64, _c_p]),
+    "ql_selftest_arm_gemm_stall": (ctypes.c_int, [ctypes.c_int, _c_i64]),
     "nf4_quantize": (ctypes.c_int, [_c_p, _c_i64, ctypes.c_int, _c_p, _c_p, _c_p]),
     "nf4_dequantize": (ctypes.c_int, [_c_p, _c_p, _c_i64, ctypes.c_int, ctypes.c_int, _c_p, _c_p]),
     "qlora_merge_lora": (ctypes.c_int, [_c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, ctypes.c_float, ctypes.c_int,
@@ -172,6 +173,12 @@ def set_profile_events(which: int, start=None, stop=None) -> None:
             ev.record()
         return ctypes.c_void_p(ev.cuda_event)
     _check(lib().ql_set_profile_events(which, handle(start), handle(stop)), "ql_set_profile_events")
+
+
+def selftest_arm_gemm_stall(role: int, wait_cycles: int) -> None:
+    """Arm the next fused GEMM launch to stall one warp role (1 MMA, 2 B producer, 3 codes producer) with every
+    wait bounded by ``wait_cycles``: a test of the kernels' abort path."""
+    _check(lib().ql_selftest_arm_gemm_stall(int(role), int(wait_cycles)), "ql_selftest_arm_gemm_stall")
 
 
 def selftest_wait_timeout(wait_cycles: int) -> None:

@@ -752,6 +752,29 @@ def run_other_workloads(peaks, dev):
             torch.cuda.empty_cache()
         except Exception as e:  # pragma: no cover - reported, never fatal for the main line
             res[name] = {"error": f"{type(e).__name__}: {e}"[:200]}
+    # The decode layer on double-quantized NF4 constants (8-bit E4M3 codes, an fp32 scale per 256 and an offset
+    # instead of fp32 absmax): the fused GEMM reads the compressed constants, so its algorithmic bytes drop by
+    # 11 MB; the fraction is taken against those bytes.
+    try:
+        w = I.WORKLOADS["decode_16x8192x28672_r16"]
+        d = I.make_linear_inputs(w)
+        wt = ops.Weight.nf4_dq(torch.from_numpy(d["W"]).to(dev))
+        A, B, x = d["A"].to(dev), d["B"].to(dev), d["x"].to(dev)
+        M, N, K, r = w.M, w.N, w.K, w.r
+        f_ms = timeit(lambda: ops.linear_fwd_w(x, wt, A, B, w.s))
+        k_ms = kernel_ms(lambda: ops.linear_fwd_w(x, wt, A, B, w.s), 0)
+        nb = N * K // 64
+        dq_bytes = N * K // 2 + nb + (nb + 255) // 256 * 4 + 4 + 2 * M * K + 2 * M * N + 2 * r * K + 2 * N * r
+        res["decode_16x8192x28672_r16_nf4dq"] = {
+            "fwd_ms": round(f_ms, 4), "fwd_gbs": round(dq_bytes / (f_ms * 1e-3) / 1e9, 1),
+            "fwd_roofline_frac": round(dq_bytes / (f_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "fused_fwd_ms": round(k_ms, 4),
+            "fused_fwd_hbm_frac": round(dq_bytes / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "algorithmic_bytes": int(dq_bytes), "nf4_algorithmic_bytes": int(w.bytes_fwd)}
+        del wt, A, B, x, d
+        torch.cuda.empty_cache()
+    except Exception as e:  # pragma: no cover - reported, never fatal for the main line
+        res["decode_16x8192x28672_r16_nf4dq"] = {"error": f"{type(e).__name__}: {e}"[:200]}
     # The NVFP4 form of the layer on the block-scaled FP4 tensor core: the layer forward (activation quantization,
     # s x A^T, the FP4 GEMM) and the FP4 GEMM alone.  Its peak is the measured bf16 peak times 4, the ratio of
     # the nominal dense FP4 and bf16 tensor rates (9 and 2.25 PFLOP/s).

@@ -488,7 +488,12 @@ def run_ours_linear(args, rank, world, local, peaks):
         d["x"] = I.draw_x(I._streams(1000 + rank), w.M, w.K, w.x_kind)
         d["dy"] = I.draw_dy(w.M, w.N, 2000 + rank)
     dev = torch.device("cuda", local)
-    layer = ops.QLoRALinear(torch.from_numpy(d["W"]).to(dev), d["A"].to(dev), d["B"].to(dev), d["s"])
+    if args.fp4:  # the NVFP4 form on the block-scaled FP4 tensor core: forward only
+        import dataclasses
+        w = dataclasses.replace(w, backward=False)
+        layer = ops.FP4Linear(torch.from_numpy(d["W"]).to(dev), d["A"].to(dev), d["B"].to(dev), d["s"])
+    else:
+        layer = ops.QLoRALinear(torch.from_numpy(d["W"]).to(dev), d["A"].to(dev), d["B"].to(dev), d["s"])
     x = d["x"].to(dev)
     dy = d["dy"].to(dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
@@ -540,7 +545,13 @@ def run_ours_linear(args, rank, world, local, peaks):
         kern["fused_dx"] = {"ms": sum(e[4].elapsed_time(e[5]) for e in ev) / K, "flops": 2 * M * N * Kd + 2 * M * Kd * r}
     dom = max(kern, key=lambda k: kern[k]["ms"])
     traffic = load_traffic(w.name).get(dom)
-    if w.backward:
+    if args.fp4:
+        ach = kern[dom]["flops"] / (kern[dom]["ms"] * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "fp4_gemm", "achieved": round(ach, 1), "peak": 4 * peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": round(ach / (4 * peaks["bf16_tflops"]), 4),
+                    "peak_source": peaks["source"] + " bf16 burst x 4 (nominal dense FP4 / bf16 ratio)",
+                    "traffic": load_traffic(w.name + "_fp4").get("fp4_gemm"), "kernel_ms": round(kern[dom]["ms"], 4)}
+    elif w.backward:
         ach = kern[dom]["flops"] / (kern[dom]["ms"] * 1e-3) / 1e12
         roofline = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4),
@@ -556,8 +567,9 @@ def run_ours_linear(args, rank, world, local, peaks):
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "M": M, "N": N, "K": Kd, "r": r, "s": w.s, "tokens_per_rank": M,
+        "vs_baseline": None, "dtype": "e2m1" if args.fp4 else "bf16", "data": "synthetic",
+        "config": {"workload": w.name + ("_fp4" if args.fp4 else ""), "M": M, "N": N, "K": Kd, "r": r, "s": w.s,
+                   "tokens_per_rank": M,
                    "global_tokens": M * world, "parallelism": f"dp{world}",
                    "l2": "flushed before every timed step (256 MiB write, outside the timed interval)"},
         "roofline": roofline,
@@ -575,6 +587,56 @@ E2E_RESULTS = {
     # every output of the step
     "all": ("y", "dx", "dA", "dB"),
 }
+
+
+def run_e2e_fp4(ctx, args, world):
+    """The NVFP4 forward through its public call with host buffers: x copied in, y read back, pipelined as the
+    other end-to-end measurements."""
+    import torch
+
+    layer, _x, _dy, d, w, dev = ctx
+    x_h = d["x"].pin_memory()
+    M, N = w.M, w.N
+    slots = [dict(x=torch.empty_like(d["x"], device=dev), y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                  h=torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True), ready=torch.cuda.Event(),
+                  done=torch.cuda.Event(), out=torch.cuda.Event()) for _ in range(2)]
+    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def issue(i):
+        sl = slots[i % 2]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(sl["done"])
+            sl["x"].copy_(x_h, non_blocking=True)
+            sl["ready"].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(sl["ready"])
+            if i >= 2:
+                s_comp.wait_event(sl["out"])
+            layer.forward(sl["x"], y=sl["y"])
+            sl["done"].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(sl["done"])
+            sl["h"].copy_(sl["y"], non_blocking=True)
+            sl["out"].record(s_out)
+
+    for i in range(max(args.warmup, 3)):
+        issue(i)
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for i in range(args.steps):
+        issue(i)
+    for st in (s_in, s_comp):
+        ev = torch.cuda.Event()
+        ev.record(st)
+        s_out.wait_event(ev)
+    end.record(s_out)
+    torch.cuda.synchronize(dev)
+    total = max_over_ranks(start.elapsed_time(end), world)
+    val = w.flops_fwd * world * args.steps / (total * 1e-3) / 1e12
+    return {"value": round(val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(M * w.K * 2),
+            "d2h_bytes_per_step": int(M * N * 2), "ms_per_step": round(total / args.steps, 4), "read_back": "y"}
 
 
 def run_e2e_linear(ctx, args, world, read_back: str = "grads"):
@@ -1017,6 +1079,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--only-main", action="store_true", help="skip the other workloads and the CPU baseline")
     ap.add_argument("--ref-tokens", type=int, default=CHAIN_SAMPLE_TOKENS, help="tokens per oracle step (reference arm)")
+    ap.add_argument("--fp4", action="store_true",
+                    help="with a single-layer --workload: its NVFP4 forward on the block-scaled FP4 tensor core")
     ap.add_argument("--tokens", type=int, default=None,
                     help="token batch of the gated-MLP block (default 8192; smaller batches are for profiler captures)")
     args = ap.parse_args()
@@ -1039,7 +1103,7 @@ def main():
         dev = ctx[3]
     else:
         out, ctx = run_ours_linear(args, rank, world, local, peaks)
-        out["e2e"] = run_e2e_linear(ctx, args, world, "grads")
+        out["e2e"] = run_e2e_fp4(ctx, args, world) if args.fp4 else run_e2e_linear(ctx, args, world, "grads")
         if ctx[4].backward:
             full = run_e2e_linear(ctx, args, world, "all")
             out["e2e"]["all_outputs"] = {k: full[k] for k in ("value", "ms_per_step", "d2h_bytes_per_step",

@@ -35,8 +35,8 @@
 // Warp roles: warp 0 = B producer (lane 0 issues TMA), warp 1 = TMEM allocator + MMA issuer, warps 2..5 =
 // epilogue (TMEM -> registers -> global), warps 6 .. 6 + 4G - 1 = dequantizers (G groups of 4 warps; group
 // g % G takes stage g), warp 6 + 4G = Q producer (lane 0 issues the codes TMA, all lanes copy absmax), and in
-// the fused SwiGLU forward four more epilogue warps after it (each epilogue warp then drains half the
-// columns of its lane quarter).  The dequantizer and Q-producer warps exist in the dequantizing modes only.
+// the tensor-memory forward at BN >= 128 four more epilogue warps after it (each epilogue warp then drains
+// half the columns of its lane quarter).  The dequantizer and Q-producer warps exist in the dequantizing modes only.
 //
 // Shared-memory tiles: for the 128B swizzle every tile starts on a 1024-byte boundary; row r of a tile is
 // 128 bytes at r*128 and its 16-byte chunk c sits at chunk position c ^ (r & 7).  TMA writes that layout;
@@ -229,10 +229,11 @@ struct UmmaCfg {
   // spends most of a stage waiting on its own instruction latencies, so stage throughput grows with the
   // number of groups in flight, up to the A ring's depth: 4 in the TMEM kernel, 3 in the MN-major one.
   static constexpr int kDeqWarpsPerGroup = 4;
-  // The fused SwiGLU forward epilogue is long and, with one accumulator at BN >= 128, not overlapped with the
-  // next unit's MMAs: it runs on 8 epilogue warps (two per lane quarter, each draining half the columns), and
-  // its CTA has one dequantizer group fewer to stay within the register file.
-  static constexpr int kEpiWarps = (EPI == EPI_SWIGLU_FWD && BN >= 128) ? 8 : 4;
+  // The forward at BN >= 128 keeps A in tensor memory, which leaves room for one accumulator only, so its
+  // epilogue (the fused SwiGLU one above all) is not overlapped with the next unit's MMAs: it runs on 8 epilogue
+  // warps (two per lane quarter, each draining half the columns), and the CTA has one dequantizer group fewer
+  // to stay within the register file.
+  static constexpr int kEpiWarps = (AM == A_DEQ_TMEM && BN >= 128) ? 8 : 4;
   static constexpr int kDeqCap = kATmem ? (kEpiWarps == 8 ? 3 : 4) : 3;
   static constexpr int kDeqGroups = kDeq ? (kAStages < kDeqCap ? kAStages : kDeqCap) : 0;
   static constexpr int kQWarp = 6 + 4 * kDeqGroups;

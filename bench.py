@@ -13,8 +13,8 @@ own batch (data parallel, weak scaling) and the adapter gradients are summed ove
 are quantized once before timing (they are frozen), as in fine-tuning.
 
 Timing: W warm-up steps, then K steps, each bracketed by CUDA events on the launching stream; the L2 is flushed
-(256 MiB write) before every step outside the timed interval; barrier + synchronize on both sides of the timed
-loop; the result is the max over ranks.  rank 0 prints one JSON line.
+(256 MiB written, then read back so that L2 holds clean lines) before every step outside the timed interval;
+barrier + synchronize on both sides of the timed loop; the result is the max over ranks.  rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle (the only reference that exists for these layers) on a bounded sample
 of the same workload, on the host cores, rank 0 only.
@@ -201,7 +201,12 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 def flush_l2(buf):
+    """Evict the workload from L2: write a 256 MiB buffer, then read it back.  The read leaves L2 holding clean
+    lines of the flush buffer, so the timed kernels do not pay for writing the flush's dirty lines back to HBM
+    (on a B200 that write-back cost a 30 us, 132 MB streaming kernel about 8 us)."""
+    import torch
     buf.zero_()
+    buf.view(torch.int32).sum(dtype=torch.int64)
 
 
 # ------------------------------------------------------------------------------------------ work per workload
@@ -375,7 +380,7 @@ def run_ours_chain(args, rank, world, local, peaks):
         "config": {"workload": CHAIN_WORKLOAD, "M": M, "D": D, "F": F, "r": r, "s": 2.0, "tokens_per_rank": M,
                    "global_tokens": M * world, "parallelism": f"dp{world}",
                    "layers": "gate+up (stacked, SwiGLU in the epilogue) and down, NF4 block 64, one LoRA pair each",
-                   "l2": "flushed before every timed step (256 MiB write, outside the timed interval); inputs "
+                   "l2": "flushed before every timed step (256 MiB written, then read back; outside the timed interval); inputs "
                          "(134 MB activations, 396 MB of NF4 weights) exceed the 126 MB L2"},
         "roofline": roofline,
         "step_roofline_frac": round(step_roof_ms / ms_per_step, 4),
@@ -571,7 +576,7 @@ def run_ours_linear(args, rank, world, local, peaks):
         "config": {"workload": w.name + ("_fp4" if args.fp4 else ""), "M": M, "N": N, "K": Kd, "r": r, "s": w.s,
                    "tokens_per_rank": M,
                    "global_tokens": M * world, "parallelism": f"dp{world}",
-                   "l2": "flushed before every timed step (256 MiB write, outside the timed interval)"},
+                   "l2": "flushed before every timed step (256 MiB written, then read back; outside the timed interval)"},
         "roofline": roofline,
         "step_roofline_frac": round(step_roof_ms / ms_per_step, 4),
         "gpu_launches": int(launches),

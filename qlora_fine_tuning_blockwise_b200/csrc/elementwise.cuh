@@ -9,35 +9,39 @@
 
 namespace qlora {
 
-// Midpoints between adjacent levels, exact in fp64 (a sum of two fp32 values and a halving).
-__constant__ double kNF4Mid[15] = {
-    (double(kNF4Levels[0]) + double(kNF4Levels[1])) * 0.5,   (double(kNF4Levels[1]) + double(kNF4Levels[2])) * 0.5,
-    (double(kNF4Levels[2]) + double(kNF4Levels[3])) * 0.5,   (double(kNF4Levels[3]) + double(kNF4Levels[4])) * 0.5,
-    (double(kNF4Levels[4]) + double(kNF4Levels[5])) * 0.5,   (double(kNF4Levels[5]) + double(kNF4Levels[6])) * 0.5,
-    (double(kNF4Levels[6]) + double(kNF4Levels[7])) * 0.5,   (double(kNF4Levels[7]) + double(kNF4Levels[8])) * 0.5,
-    (double(kNF4Levels[8]) + double(kNF4Levels[9])) * 0.5,   (double(kNF4Levels[9]) + double(kNF4Levels[10])) * 0.5,
-    (double(kNF4Levels[10]) + double(kNF4Levels[11])) * 0.5, (double(kNF4Levels[11]) + double(kNF4Levels[12])) * 0.5,
-    (double(kNF4Levels[12]) + double(kNF4Levels[13])) * 0.5, (double(kNF4Levels[13]) + double(kNF4Levels[14])) * 0.5,
-    (double(kNF4Levels[14]) + double(kNF4Levels[15])) * 0.5,
-};
-
-// Code of a normalised value: binary search for the number of midpoints strictly below n (exact fp64
-// comparisons; a value equal to a midpoint counts that midpoint as not below, so ties take the lower code).
-__device__ __forceinline__ uint32_t nf4_code(float n) {
-  const double v = static_cast<double>(n);
-  uint32_t lo = 0;  // answer in [0, 15]
+// Code of a normalised value n: the number of midpoints m_i = (L_i + L_{i+1}) / 2 (exact in fp64) strictly below
+// n, so a value equal to a midpoint takes the lower code.  For an fp32 n, "n > m_i" is the same test as
+// "n >= t_i" with t_i the least fp32 value above m_i (m_i rounded up to fp32, stepped once more when m_i is
+// itself an fp32 value), so the fifteen comparisons run in fp32 against per-thread register thresholds, and a
+// four-level branch-free search (each level picks the next threshold by select) finds the count.  A NaN fails
+// every comparison and takes code 0, as it fails every "n > m_i".
+struct Nf4Thresholds {
+  float t[15];
+  __device__ __forceinline__ Nf4Thresholds() {
 #pragma unroll
-  for (uint32_t step = 8; step > 0; step >>= 1) {
-    // invariant: midpoints [0, lo) are below v; test midpoint lo + step - 1
-    if (lo + step <= 15 && v > kNF4Mid[lo + step - 1]) lo += step;
+    for (int i = 0; i < 15; ++i) {
+      const double m = (static_cast<double>(kNF4LevelsDev[i]) + static_cast<double>(kNF4LevelsDev[i + 1])) * 0.5;
+      const float up = __double2float_ru(m);
+      t[i] = static_cast<double>(up) == m ? nextafterf(up, INFINITY) : up;
+    }
   }
-  return lo;
-}
+  __device__ __forceinline__ uint32_t code(float n) const {
+    const bool b3 = n >= t[7];
+    const bool b2 = n >= (b3 ? t[11] : t[3]);
+    const bool b1 = n >= (b3 ? (b2 ? t[13] : t[9]) : (b2 ? t[5] : t[1]));
+    const float t0 = b3 ? (b2 ? (b1 ? t[14] : t[12]) : (b1 ? t[10] : t[8]))
+                        : (b2 ? (b1 ? t[6] : t[4]) : (b1 ? t[2] : t[0]));
+    const bool b0 = n >= t0;
+    return (static_cast<uint32_t>(b3) << 3) | (static_cast<uint32_t>(b2) << 2) | (static_cast<uint32_t>(b1) << 1) |
+           static_cast<uint32_t>(b0);
+  }
+};
 
 // One warp per 64-element block: lane l owns elements 2l, 2l+1 (one packed byte).
 __global__ void nf4_quantize_kernel(const float* __restrict__ w, long long nblocks, uint8_t* __restrict__ codes,
                                     float* __restrict__ absmax, unsigned int* err) {
   const int lane = threadIdx.x & 31;
+  const Nf4Thresholds thr;
   const long long warps_total = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   for (long long b = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); b < nblocks;
        b += warps_total) {
@@ -49,8 +53,8 @@ __global__ void nf4_quantize_kernel(const float* __restrict__ w, long long nbloc
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, kDevErrNonFinite);
     uint32_t c0 = 7, c1 = 7;
     if (m > 0.0f) {
-      c0 = nf4_code(__fdiv_rn(v.x, m));
-      c1 = nf4_code(__fdiv_rn(v.y, m));
+      c0 = thr.code(__fdiv_rn(v.x, m));
+      c1 = thr.code(__fdiv_rn(v.y, m));
     }
     codes[b * 32 + lane] = static_cast<uint8_t>((c0 << 4) | c1);
     if (lane == 0) absmax[b] = m;
@@ -75,6 +79,7 @@ __global__ void lora_merge_kernel(const uint8_t* __restrict__ codes, const float
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int kb = K / 64;
+  const Nf4Thresholds thr;
   const long long warps_total = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   for (long long b = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); b < nblocks;
        b += warps_total) {
@@ -107,8 +112,8 @@ __global__ void lora_merge_kernel(const uint8_t* __restrict__ codes, const float
       if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, kDevErrNonFinite);
       uint32_t c0 = 7, c1 = 7;
       if (m > 0.0f) {
-        c0 = nf4_code(__fdiv_rn(w0, m));
-        c1 = nf4_code(__fdiv_rn(w1, m));
+        c0 = thr.code(__fdiv_rn(w0, m));
+        c1 = thr.code(__fdiv_rn(w1, m));
       }
       codes_out[b * 32 + lane] = static_cast<uint8_t>((c0 << 4) | c1);
       if (lane == 0) absmax_out[b] = m;
@@ -116,37 +121,42 @@ __global__ void lora_merge_kernel(const uint8_t* __restrict__ codes, const float
   }
 }
 
-// Each thread expands 8 elements (4 code bytes) with one absmax.
+// Each thread expands 32 elements (16 code bytes, half a block) with one absmax: one 16-byte load of codes and
+// 64 (bf16) or 128 (fp32) bytes of 16-byte stores, so every thread keeps a whole vector of HBM reads in flight.
 template <bool kBf16>
 __global__ void nf4_dequantize_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ absmax,
-                                      long long ngroups, void* __restrict__ out) {
+                                      long long nhalves, void* __restrict__ out) {
   __shared__ float lv[16];
   if (threadIdx.x < 16) lv[threadIdx.x] = kNF4LevelsDev[threadIdx.x];
   __syncthreads();
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
-    const uint32_t wv = __ldg(reinterpret_cast<const uint32_t*>(codes) + g);
-    const float sc = __ldg(absmax + (g >> 3));  // 8 groups of 8 per 64-element block
-    float f[8];
+  for (long long q = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; q < nhalves; q += stride) {
+    const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes) + q);
+    const float sc = __ldg(absmax + (q >> 1));
+    const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const uint32_t byte = (wv >> (8 * b)) & 0xFFu;
-      f[2 * b] = __fmul_rn(lv[byte >> 4], sc);
-      f[2 * b + 1] = __fmul_rn(lv[byte & 15u], sc);
-    }
-    if (kBf16) {
-      uint4 o;
-      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+    for (int v = 0; v < 4; ++v) {
+      float f[8];
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * b], f[2 * b + 1]);
-        op[b] = *reinterpret_cast<uint32_t*>(&h);
+        const uint32_t byte = (w4[v] >> (8 * b)) & 0xFFu;
+        f[2 * b] = __fmul_rn(lv[byte >> 4], sc);
+        f[2 * b + 1] = __fmul_rn(lv[byte & 15u], sc);
       }
-      reinterpret_cast<uint4*>(out)[g] = o;
-    } else {
-      float4* o = reinterpret_cast<float4*>(out) + 2 * g;
-      o[0] = make_float4(f[0], f[1], f[2], f[3]);
-      o[1] = make_float4(f[4], f[5], f[6], f[7]);
+      if (kBf16) {
+        uint4 o;
+        uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * b], f[2 * b + 1]);
+          op[b] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        reinterpret_cast<uint4*>(out)[4 * q + v] = o;
+      } else {
+        float4* o = reinterpret_cast<float4*>(out) + 8 * q + 2 * v;
+        o[0] = make_float4(f[0], f[1], f[2], f[3]);
+        o[1] = make_float4(f[4], f[5], f[6], f[7]);
+      }
     }
   }
 }

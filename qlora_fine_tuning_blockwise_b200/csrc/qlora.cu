@@ -970,13 +970,13 @@ ql_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t nume
   if (blocksize != 64) return QL_ERR_UNSUPPORTED;
   DeviceInfo d;
   if (!device_info(&d)) return QL_ERR_CUDA;
-  const long long ngroups = numel / 8;
+  const long long nhalves = numel / 32;  // 32 elements (16 code bytes) per thread
   const int threads = 256;
-  const long long ctas = std::min<long long>(cdiv(ngroups, threads), static_cast<long long>(d.sms) * 16);
+  const long long ctas = std::min<long long>(cdiv(nhalves, threads), static_cast<long long>(d.sms) * 8);
   if (out_dtype == QL_BF16)
-    nf4_dequantize_kernel<true><<<static_cast<unsigned>(ctas), threads, 0, as_stream(stream)>>>(codes, absmax, ngroups, out);
+    nf4_dequantize_kernel<true><<<static_cast<unsigned>(ctas), threads, 0, as_stream(stream)>>>(codes, absmax, nhalves, out);
   else
-    nf4_dequantize_kernel<false><<<static_cast<unsigned>(ctas), threads, 0, as_stream(stream)>>>(codes, absmax, ngroups, out);
+    nf4_dequantize_kernel<false><<<static_cast<unsigned>(ctas), threads, 0, as_stream(stream)>>>(codes, absmax, nhalves, out);
   count_launch();
   return status_of(cudaGetLastError());
 }

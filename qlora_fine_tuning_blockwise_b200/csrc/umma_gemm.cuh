@@ -202,8 +202,13 @@ struct UmmaCfg {
   static constexpr int kCBytes = 4096 * KB;                       // 128 rows x 64 KB codes
   static constexpr int kSBytes = 512 * KB;                        // 128 rows x KB absmax values
   static constexpr int kQSlot = kDeq ? kCBytes + kSBytes : 0;
-  // the dequantizers look codes up in a shared-memory table of bf16 level pairs, one copy per lane (32 KB)
-  static constexpr int kLutBytes = kDeq ? 256 * 32 * 4 : 0;
+  // the dequantizers look codes up in a shared-memory table of bf16 level pairs, one copy per lane, placed at
+  // the start of the dynamic shared memory (a fixed address the compiler folds into the loads): entry stride
+  // 128 bytes (32 KB), or -- in the token-light 4-block kernels at BN <= 32, whose dequantizers bound the
+  // kernel -- entry stride 256 bytes (64 KB, half of it padding), so that one byte permute of (code byte, lane)
+  // is the whole offset
+  static constexpr bool kWideLut = kDeq && KB == 4 && BN <= 32;
+  static constexpr int kLutBytes = kDeq ? (kWideLut ? 256 * 64 * 4 : 256 * 32 * 4) : 0;
   static constexpr int kBarBytes = 1024;
   static constexpr int kBudget = 226 * 1024 - 1024 - kLutBytes - kBarBytes;
 
@@ -216,7 +221,7 @@ struct UmmaCfg {
 
   // ring depths: deep B rings when B tiles are small (token-light layers), 4 stages of 16-32 KB otherwise;
   // the A ring as deep as tensor memory (or shared memory, for A_DEQ_MN) allows.
-  static constexpr int kBStagesWant = kDeq ? (BN <= 64 ? 8 : (AM == A_DEQ_MN && BN >= 256 ? 3 : 4)) : 8;
+  static constexpr int kBStagesWant = kDeq ? (kWideLut ? 4 : BN <= 64 ? 8 : (AM == A_DEQ_MN && BN >= 256 ? 3 : 4)) : 8;
   static constexpr int kAStagesWant = kATmem ? kAStagesTmem : (AM == A_DEQ_MN ? (BN >= 256 ? 3 : 4) : 0);
   static constexpr int kQWant = KB == 4 ? 6 : (BN >= 128 ? 10 : 16);
   static constexpr int kBFit = (kBudget - kAStagesWant * kASlot - (kDeq ? kQWant * kQSlot : 0)) / kBSlot;
@@ -299,14 +304,16 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
   constexpr uint32_t kFull = 0xffffffffu;
 
   extern __shared__ uint8_t smem_raw[];
+  // the level-pair table first (at the array's own address), then the rings from the next 1024-byte boundary;
   // align by pointer arithmetic on the shared array itself (not through an integer), so every pointer derived
   // from it stays a known shared-memory pointer and compiles to shared loads and stores
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint32_t* sLut = reinterpret_cast<uint32_t*>(smem_raw);
+  uint8_t* ring_raw = smem_raw + C::kLutBytes;
+  const uint32_t raw_addr = smem_u32(ring_raw);
+  uint8_t* smem = ring_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sB = smem;                          // B ring (B, then A in the TMA modes), 1024-aligned slots
   uint8_t* sA = sB + BS * C::kBSlot;           // A ring of A_DEQ_MN, 1024-aligned slots
   uint8_t* sQ = sA + AS * C::kASlot;           // Q ring: codes, then absmax
-  uint32_t* sLut = reinterpret_cast<uint32_t*>(sQ + QS * C::kQSlot);
   // Phases: b_* advance once per stage (every stage uses the B ring), a_* once per stage in the dequantizing
   // modes, q_* once per MAIN stage, tmem_* once per unit accumulated in that buffer.  Each waiter derives
   // the parity from its running count of the ring's uses, which is sound only while the barrier's previous
@@ -316,7 +323,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
   //     a_empty wait, G = dequantizer groups), so with G <= AS its a_empty wait for stage g - AS cannot see
   //     an older phase, and with QS >= AS + G the Q stage QS before its own has been consumed;
   //   - the MMA and the producers visit every phase of the barriers they wait on, in order.
-  uint64_t* b_full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sLut) + C::kLutBytes);
+  uint64_t* b_full = reinterpret_cast<uint64_t*>(sQ + QS * C::kQSlot);
   uint64_t* b_empty = b_full + BS;
   uint64_t* a_full = b_empty + BS;
   uint64_t* a_empty = a_full + AS;
@@ -359,14 +366,15 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
     fence_mbar_init();
   }
   if constexpr (C::kLutBytes > 0) {
-    // entry (byte b, lane l) at word 32 b + l: the bf16 pair of the byte's two elements, element 2j in the low
-    // half.  NF4 bytes hold element 2j in the high nibble, NVFP4 bytes in the low nibble.
+    // entry (byte b, lane l) at word 32 b + l (64 b + l in the wide table): the bf16 pair of the byte's two
+    // elements, element 2j in the low half.  NF4 bytes hold element 2j in the high nibble, NVFP4 bytes in the
+    // low nibble.
     constexpr bool fp4 = WF == WF_NVFP4;
     for (int idx = threadIdx.x; idx < 256 * 32; idx += blockDim.x) {
       const int b = idx >> 5;
       __nv_bfloat162 h = fp4 ? __floats2bfloat162_rn(e2m1_value_dev(b & 15), e2m1_value_dev(b >> 4))
                              : __floats2bfloat162_rn(kNF4LevelsDev[b >> 4], kNF4LevelsDev[b & 15]);
-      sLut[idx] = *reinterpret_cast<uint32_t*>(&h);
+      sLut[C::kWideLut ? 64 * b + (idx & 31) : idx] = *reinterpret_cast<uint32_t*>(&h);
     }
   }
   if (warp == 0 && lane == 0) {
@@ -737,6 +745,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
       const int s_idx = C::kATmem ? row : (row * 2 + h);
       const uint32_t t_lane = static_cast<uint32_t>(32 * (warp & 3)) << 16;
       const uint8_t* lut_lane = reinterpret_cast<const uint8_t*>(sLut) + lane * 4;
+      const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
       const float dq_mu = WF == WF_NF4_DQ ? *args.dq_mu : 0.0f;
       const float fp4_S = WF == WF_NVFP4 ? *args.fp4_S : 0.0f;
       int g = 0, q = 0;
@@ -876,11 +885,14 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
               for (int w = 0; w < 8; ++w) {
                 const __nv_bfloat162 sc2 = sc2q[w >> 1];
                 const uint32_t qw8 = words[8 * p + w];
-                const uint32_t offs[4] = {(qw8 << 7) & 0x7F80u, (qw8 >> 1) & 0x7F80u, (qw8 >> 9) & 0x7F80u,
-                                          (qw8 >> 17) & 0x7F80u};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                  uint32_t v = *reinterpret_cast<const uint32_t*>(lut_lane + offs[j]);
+                  // byte offset of (code byte j, lane) in the table: one byte permute into (byte << 8) | 4 lane for
+                  // the wide table, a permute and a shift-add for the narrow one
+                  const uint32_t off =
+                      C::kWideLut ? __byte_perm(qw8, lane4, 0x5504u | (static_cast<uint32_t>(j) << 4))
+                                  : (__byte_perm(qw8, 0u, 0x4440u + static_cast<uint32_t>(j)) << 7) + lane4;
+                  uint32_t v = *reinterpret_cast<const uint32_t*>(smem_raw + off);
                   __nv_bfloat162 pr = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc2);
                   r[4 * w + j] = *reinterpret_cast<uint32_t*>(&pr);
                 }

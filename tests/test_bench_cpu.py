@@ -112,3 +112,12 @@ def test_clock_summary_parses_samples_and_reasons():
     assert c.summary()["reasons"] == ["hw_thermal_slowdown"]
     c.lines = []
     assert c.summary()["reasons"] == ["unsampled"]
+
+
+def test_flush_l2_writes_then_reads():
+    """The flush zeroes its buffer (the write that evicts the workload) and then reads it back."""
+    import torch
+    b = load_bench()
+    buf = torch.full((4096,), 7, dtype=torch.uint8)
+    b.flush_l2(buf)
+    assert int(buf.sum()) == 0

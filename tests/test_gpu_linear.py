@@ -87,6 +87,24 @@ def test_forward_backward_small(ops, M, N, K, r):
         assert_close(got["dB"], ref["dB"], "dB")
 
 
+@pytest.mark.parametrize("M,N,K,r,s", [
+    (64, 256, 256, 8, -1.5),     # BN = 64 forward, one LoRA stage
+    (300, 264, 256, 16, -2.0),   # BN = 256 forward, ragged token and weight tiles
+    (1, 264, 512, 16, -0.25),    # token-light forward in four-block stages
+    (40, 136, 768, 72, -1.0),    # two LoRA stages, partly filled
+])
+def test_negative_scaling(ops, M, N, K, r, s):
+    """A negative s flips the sign of the LoRA term in y, of v = s dY B in dX and of both adapter gradients."""
+    d = I.make_random_linear(M, N, K, r, s=s, seed=M + N + K + r + 1000)
+    got = run_gpu(ops, d)
+    ref = oracle_all(d)
+    for k, name in (("y", "y"), ("dx", "dX"), ("su", "s*x*A^T"), ("dA", "dA"), ("dB", "dB")):
+        assert_close(got[k], ref[k], f"{name} s={s}")
+    # the LoRA term really is subtracted: removing it moves y away from the reference
+    base = L.qlora_forward(f64(d["x"]), oracle_weight(d["W"]), f64(d["A"]), f64(d["B"]), 0.0)
+    assert np.linalg.norm(base - ref["y"]) > 1e-2 * np.linalg.norm(ref["y"])
+
+
 def test_backward_recomputes_su_when_not_given(ops):
     d = I.make_random_linear(96, 264, 320, 16, s=0.5, seed=11)
     a = run_gpu(ops, d, pass_su=True)

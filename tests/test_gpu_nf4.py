@@ -90,21 +90,35 @@ def test_quantize_edge_values(ops):
     check_roundtrip(ops, W)
 
 
-def test_quantize_all_fp32_in_unit_interval_sampled(ops):
-    """Every 64th fp32 bit pattern in [0, 1] and its negative, as normalised values of blocks with absmax 1."""
-    pats = np.arange(0, 0x3F800001, 64, dtype=np.uint32)
-    vals = pats.view(np.float32)
-    vals = np.concatenate([vals, -vals])
-    pad = (-vals.size) % 63
-    vals = np.concatenate([vals, np.zeros(pad, np.float32)]).reshape(-1, 63)
-    W = np.concatenate([np.ones((vals.shape[0], 1), np.float32), vals], axis=1).reshape(1, -1)
-    w = dev(W.reshape(-1))
-    codes, absmax = ops.nf4_quantize(w)
-    # expected codes: the oracle's rule applied to the normalised values (here n = w since absmax = 1)
-    exp = O.nf4_code_of(W.reshape(-1))
-    packed = ((exp[0::2] << 4) | exp[1::2]).astype(np.uint8)
-    assert np.array_equal(codes.cpu().numpy(), packed)
-    assert np.all(absmax.cpu().numpy() == 1.0)
+def test_quantize_every_fp32_in_unit_interval(ops):
+    """Every fp32 bit pattern in [0, 1] and its negative, as the normalised values of blocks whose absmax is 1
+    (one element 1.0, then 63 values), in chunks; the expected codes come from the oracle's rule on the same
+    values."""
+    top = 0x3F800000 + 1          # patterns 0 .. bits(1.0)
+    chunk = 63 * (1 << 19)        # whole blocks of 63 values
+    one = int(O.nf4_code_of(np.array([1.0], np.float32))[0])
+    for p0 in range(0, top, chunk):
+        p1 = min(p0 + chunk, top)
+        n = p1 - p0
+        nb = -(-n // 63)
+        host = np.arange(p0, p1, dtype=np.uint32).view(np.float32)
+        pats = torch.arange(p0, p1, dtype=torch.int64, device="cuda").to(torch.int32).view(torch.float32)
+        for sign in (1.0, -1.0):
+            v = torch.zeros(nb * 63, dtype=torch.float32, device="cuda")
+            v[:n] = pats * sign
+            W = torch.cat([torch.ones(nb, 1, dtype=torch.float32, device="cuda"), v.view(nb, 63)], dim=1)
+            codes, absmax = ops.nf4_quantize(W.reshape(-1).contiguous())
+            vh = np.zeros(nb * 63, np.float32)
+            vh[:n] = host * np.float32(sign)
+            e = O.nf4_code_of(vh).reshape(nb, 63).astype(np.uint8)
+            full = np.concatenate([np.full((nb, 1), one, np.uint8), e], axis=1)
+            packed = ((full[:, 0::2] << 4) | full[:, 1::2]).astype(np.uint8).reshape(-1)
+            got = codes.cpu().numpy()
+            if not np.array_equal(got, packed):
+                bad = int(np.flatnonzero(got != packed)[0])
+                raise AssertionError(f"chunk {p0:#x} sign {sign}: first differing code byte {bad}")
+            assert bool((absmax == 1.0).all())
+    assert ops.device_error() == ops.QL_OK
 
 
 def test_dequantize_ragged_sizes(ops):

@@ -189,6 +189,7 @@ struct GemmCall {
   int splits = 1;
   int prof = -1;          // profiling-event slot recorded around this launch (-1: none)
   int ctas = 0;           // persistent CTAs: at most one per SM (0: as many as the GPU has SMs)
+  bool streamk = false;   // stream-K schedule (one tile column; fp32 partial slabs reduced afterwards)
   UmmaArgs args{};
 };
 
@@ -239,7 +240,9 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
   auto kern = umma_gemm_kernel<BN, AM, BMN, KB, PAIR, WF, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int64_t units = static_cast<int64_t>(g.args.splits) * g.args.tiles_i * g.args.tiles_j;
+  // work items that size the grid: units, or with stream-K the stages of the whole sequence
+  const int64_t units = g.args.sk_stages > 0 ? static_cast<int64_t>(g.args.tiles_i) * g.args.sk_stages
+                                             : static_cast<int64_t>(g.args.splits) * g.args.tiles_i * g.args.tiles_j;
   if constexpr (PAIR) {
     // clusters of two CTAs, each pair walking the units; no more pairs than can be resident at once (a GPC with
     // an odd number of free SMs leaves one idle), so no unit waits for a pair to retire
@@ -447,6 +450,7 @@ int fwd_stage_blocks(int64_t M, int64_t K) { return (main_bn(M) <= 64 && K % 256
 
 struct LinearPlan {
   int bn_main = 16, s_main = 1;      // forward y / backward dX
+  int sk_ctas = 0, sk_slabs = 0;     // stream-K forward: CTAs and partial slabs (0: split plan)
   int s_su = 1, s_v = 1, s_da = 1, s_db = 1;
   size_t off_su = 0, off_v = 0, off_part = 0, total = 0;
 };
@@ -461,6 +465,21 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass)
   const int64_t main_kst = pass == QL_PASS_FWD ? cdiv(K, 64 * fwd_stage_blocks(M, K)) : cdiv(N, 64);
   p.s_main = M <= 64 ? plan_splits_streaming(main_tiles, main_kst, sms) : plan_splits(main_tiles, main_kst, sms);
   size_t part = 0;
+  if (pass == QL_PASS_FWD && M <= 64) {
+    // token-light forward: a stream-K schedule balances the stages exactly (each CTA gets T / P of them, at
+    // least 4) where whole split units would leave the last wave partly empty
+    const int64_t T = main_tiles * main_kst;
+    const int64_t P = std::min<int64_t>(sms, cdiv(T, 4));
+    const int64_t split_cost = cdiv(main_tiles * p.s_main, sms) * cdiv(main_kst, p.s_main);
+    if (main_kst >= 8 && cdiv(T, P) < split_cost) {
+      p.sk_ctas = static_cast<int>(P);
+      for (int64_t t = 0; t < main_tiles; ++t)
+        p.sk_slabs = std::max<int>(p.sk_slabs, static_cast<int>(sk_cta_of(t * main_kst + main_kst - 1, T, P) -
+                                                                 sk_cta_of(t * main_kst, T, P) + 1));
+      p.s_main = 1;
+      part = std::max(part, static_cast<size_t>(p.sk_slabs) * M * N * 4);
+    }
+  }
   if (p.s_main > 1) part = std::max(part, static_cast<size_t>(p.s_main) * M * (pass == QL_PASS_FWD ? N : K) * 4);
   if (r > 0) {
     p.s_su = plan_splits(cdiv(M, 128) * (rp / rp), cdiv(K, 64), sms);
@@ -547,6 +566,27 @@ cudaError_t run_gemm(GemmCall g, void* out, bool out_bf16, float alpha, int64_t 
   g.args.cols_lim = static_cast<int>(cols_lim);
   g.args.err = err;
   g.args.group_i = unit_group(g);
+  if (g.streamk) {
+    // stream-K: every unit writes its fp32 partial to the slab of its place among the CTAs sharing its tile,
+    // then one reduction sums each tile's slabs in that order (D rows must be the fastest output index)
+    if (ls != 1 || g.args.tiles_j != 1 || !part) return cudaErrorInvalidValue;
+    const int64_t T = static_cast<int64_t>(g.args.tiles_i) * g.args.k_stages;
+    g.ctas = static_cast<int>(std::min<int64_t>(g.ctas, T));
+    g.args.sk_stages = g.args.k_stages;
+    g.args.group_i = 0;
+    g.args.out = part;
+    g.args.out_bf16 = 0;
+    g.args.alpha = 1.0f;
+    g.args.split_stride = count;
+    cudaError_t e = launch_gemm(g, stream);
+    if (e != cudaSuccess) return e;
+    const int threads = 256;
+    const int64_t blocks = std::min<int64_t>(cdiv(count, threads), 148 * 16);
+    reduce_streamk_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        part, count, count, cs, g.args.k_stages, T, g.ctas, alpha, out, out_bf16 ? 1 : 0);
+    count_launch();
+    return cudaGetLastError();
+  }
   if (g.splits == 1) {
     g.args.out = out;
     g.args.out_bf16 = out_bf16 ? 1 : 0;
@@ -695,6 +735,10 @@ ql_status linear_fwd_impl(int64_t M, int64_t N, int64_t K, int64_t r, const uint
   g.cols = M;
   g.k_total = K;
   g.splits = p.s_main;
+  if (p.sk_slabs > 0 && !epi) {
+    g.streamk = true;
+    g.ctas = p.sk_ctas;
+  }
   g.prof = 0;
   if (epi) {
     g.args.epi = epi->mode;
@@ -1035,9 +1079,10 @@ ql_status qlora_gate_up_fwd_swiglu(int64_t M, int64_t F, int64_t K, int64_t r, c
   const int64_t N = 2 * F;
   const ql_weight w = nf4_weight(codes, absmax);
   if (check_linear(M, N, K, r) != QL_OK) return QL_ERR_INVALID_ARG;
-  // the fused epilogue runs in unsplit GEMMs with one-block stages; token-light layers (4-block stages) and
-  // split contractions write gu first and run the SwiGLU as its own kernel
-  if (M > 0 && plan_linear(M, N, K, r, QL_PASS_FWD).s_main == 1 && fwd_stage_blocks(M, K) == 1) {
+  // the fused epilogue runs in unsplit GEMMs with one-block stages; token-light layers (4-block stages or a
+  // stream-K schedule) and split contractions write gu first and run the SwiGLU as its own kernel
+  const LinearPlan pl = M > 0 ? plan_linear(M, N, K, r, QL_PASS_FWD) : LinearPlan{};
+  if (M > 0 && pl.s_main == 1 && pl.sk_slabs == 0 && fwd_stage_blocks(M, K) == 1) {
     EpiArgs e;
     e.mode = EPI_SWIGLU_FWD;
     e.out2 = h;
@@ -1371,7 +1416,8 @@ bool load_forward_kernels() {
          load_umma<16, A_DEQ_TMEM, false, 4>() &&
          load_umma<32, A_DEQ_TMEM, false, 4>() && load_umma<64, A_DEQ_TMEM, false, 4>() &&
          load_umma<64, A_TMA_K, false>() && load_umma<128, A_TMA_K, false>() && load_umma<256, A_TMA_K, false>() &&
-         cudaFuncGetAttributes(&a, reduce_splits_kernel) == cudaSuccess;
+         cudaFuncGetAttributes(&a, reduce_splits_kernel) == cudaSuccess &&
+         cudaFuncGetAttributes(&a, reduce_streamk_kernel) == cudaSuccess;
 }
 
 // Contexts in which the forward's kernels have been loaded (set-up runs once per context, with the device

@@ -127,6 +127,11 @@ struct UmmaArgs {
   // within a group, so that one wave of CTAs shares a few activation tiles and a group of weight tiles and
   // both stay in L2; 0 keeps tile columns fastest
   int group_i;
+  // stream-K (token-light forward, tiles_j == 1): sk_stages > 0 is the number of stages of one tile; CTA c of the
+  // P in the grid takes stages [T c / P, T (c + 1) / P) of the sequence tile 0's stages, tile 1's, ... (T =
+  // tiles_i sk_stages), one unit per tile it touches, and writes each unit's fp32 partial to slab z = the unit's
+  // place among the CTAs sharing that tile (splits and group_i unused)
+  int sk_stages;
   int epi;
   void* out2;
   long long ls2, cs2;
@@ -140,6 +145,56 @@ struct Unit {
   int main_begin, n_main, n_extra, n_total;
 };
 
+// Stream-K: the CTA whose share holds stage x of the sequence, max{c : floor(c T / P) <= x}.
+__host__ __device__ __forceinline__ long long sk_cta_of(long long x, long long T, long long P) {
+  return ((x + 1) * P - 1) / T;
+}
+
+// Stream-K: units (tiles touched) of CTA c of P.
+__host__ __device__ __forceinline__ int sk_units(const UmmaArgs& a, long long c, long long P) {
+  const long long S = a.sk_stages, T = static_cast<long long>(a.tiles_i) * S;
+  const long long s0 = T * c / P, s1 = T * (c + 1) / P;
+  return s1 > s0 ? static_cast<int>((s1 - 1) / S - s0 / S + 1) : 0;
+}
+
+// Stream-K: unit u of CTA c of P -- the part of tile s0 / S + u inside the CTA's share, its slab z (the CTA's
+// place among those sharing the tile) and, for the part that starts the tile, the LoRA stages.
+__host__ __device__ __forceinline__ Unit sk_unit(const UmmaArgs& a, long long c, long long P, int u) {
+  Unit U;
+  const long long S = a.sk_stages, T = static_cast<long long>(a.tiles_i) * S;
+  const long long s0 = T * c / P, s1 = T * (c + 1) / P;
+  const long long t = s0 / S + u;
+  const long long b = (s0 > t * S ? s0 : t * S) - t * S, e = (s1 < (t + 1) * S ? s1 : (t + 1) * S) - t * S;
+  U.z = static_cast<int>(c - sk_cta_of(t * S, T, P));
+  U.i0 = static_cast<int>(t) * 128;
+  U.j0 = 0;
+  U.main_begin = static_cast<int>(b);
+  U.n_main = static_cast<int>(e - b);
+  U.n_extra = b == 0 ? a.n_extra : 0;
+  U.n_total = U.n_extra + U.n_main;
+  return U;
+}
+
+// Stream-K reduction: out[e] = alpha * (sum over the n(t) partial slabs of the tile t holding e, in slab order),
+// with e = j * cs + i (i the D row, fastest), t = i / 128 and n(t) the number of CTAs whose share of the stage
+// sequence (S stages per tile, T in all, P CTAs) touches tile t.  Slabs past n(t) are never read.
+__global__ void reduce_streamk_kernel(const float* __restrict__ ws, long long slab, long long count, long long cs,
+                                      long long S, long long T, long long P, float alpha, void* __restrict__ out,
+                                      int out_bf16) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < count; e += stride) {
+    const long long t = (e % cs) / 128;
+    const int n = static_cast<int>(sk_cta_of(t * S + S - 1, T, P) - sk_cta_of(t * S, T, P) + 1);
+    float acc = 0.0f;
+    for (int z = 0; z < n; ++z) acc += ws[z * slab + e];
+    acc *= alpha;
+    if (out_bf16)
+      reinterpret_cast<__nv_bfloat16*>(out)[e] = __float2bfloat16_rn(acc);
+    else
+      reinterpret_cast<float*>(out)[e] = acc;
+  }
+}
+
 // Unit u -> (split z, tile row ti, tile column tj).  Splits are outermost.  Within a split, either tile columns
 // run fastest (neighbouring units share the weight tile), or -- with group_i > 0 -- the tile rows come in groups
 // of group_i (the last group may be smaller) and within a group the rows run fastest: a wave of consecutive
@@ -147,6 +202,7 @@ struct Unit {
 // once per wave instead of the whole activation matrix being streamed again by every wave.
 // With CTA pairs a tile row is 256 weight rows and CTA `rank` of the pair owns rows 128 rank .. 128 rank + 127.
 __device__ __forceinline__ Unit unit_of(const UmmaArgs& a, int u, int BN, int pair = 1, int rank = 0) {
+  if (a.sk_stages > 0) return sk_unit(a, blockIdx.x, gridDim.x, u);  // unit u of this CTA's stream-K share
   Unit U;
   int tj, ti;
   if (a.cred > 1) {  // the S consecutive units of a cluster are the S splits of one tile
@@ -336,13 +392,14 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_units = args.splits * args.tiles_i * args.tiles_j;
+  const bool streamk = args.sk_stages > 0;
   const long long lim = args.wait_limit > 0 ? args.wait_limit : kWaitTimeoutCycles;
   // CTA pairs: the even CTA of the cluster (rank 0) is the leader -- it issues the pair's MMAs, and its barriers
   // gather both CTAs' arrivals; each pair walks the units together
   const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
-  const int first_unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int unit_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int first_unit = streamk ? 0 : PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int unit_step = streamk ? 1 : PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int num_units = streamk ? sk_units(args, blockIdx.x, gridDim.x) : args.splits * args.tiles_i * args.tiles_j;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < BS; ++s) {

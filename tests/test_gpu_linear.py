@@ -71,6 +71,10 @@ SMALL = [
     (1, 264, 512, 16),      # BN = 16, ragged N tile
     (40, 136, 768, 72),     # BN = 64, odd number of 4-block stages, partly filled LoRA stage
     (20, 128, 1280, 256),   # BN = 32, largest rank in one 256-wide LoRA stage
+    # token-light layers deep enough for the stream-K schedule (tiles shared by consecutive CTAs, fp32 slabs)
+    (16, 1024, 4096, 16),   # 4-block stages, four CTAs per tile
+    (40, 2056, 2048, 72),   # BN = 64, ragged weight tile, two CTAs per tile
+    (8, 1024, 2112, 8),     # K % 256 != 0: one-block stages
 ]
 
 

@@ -164,6 +164,8 @@ __global__ void nf4_dequantize_kernel(const uint8_t* __restrict__ codes, const f
 // out[e] = alpha * sum_s ws[s * slab + e]  (fp32 sum in split order: deterministic)
 __global__ void reduce_splits_kernel(const float* __restrict__ ws, long long slab, int nsplit, long long count,
                                      float alpha, void* __restrict__ out, int out_bf16) {
+  griddep_launch_dependents();
+  griddep_wait();  // the partials are the GEMM's output
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < count; e += stride) {
     float acc = 0.0f;

@@ -96,6 +96,19 @@ __device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, v
   }
 }
 
+// ------------------------------------------------------------------------------------------ dependent launch
+//
+// A kernel launched with programmatic stream serialization may start while the kernel before it in the stream is
+// still running.  It must call griddep_wait() before it reads anything that kernel writes, or writes anything that
+// kernel reads; griddep_launch_dependents() lets the next such kernel start early.  Both are no-ops in a kernel
+// launched the ordinary way.
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* tm) {

@@ -51,6 +51,11 @@ void prof_record(int which, int edge, cudaStream_t stream) {
   if (ev) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), stream);
 }
 
+// Whether events are set for slot `which` (a kernel timed alone is launched the ordinary way).
+bool prof_active(int which) {
+  return which >= 0 && g_prof_events[which][0].load(std::memory_order_relaxed) != nullptr;
+}
+
 int g_dev_sms[kMaxDevices] = {};
 cudaStream_t g_dev_side[kMaxDevices] = {};
 std::mutex g_dev_mu;
@@ -190,8 +195,28 @@ struct GemmCall {
   int prof = -1;          // profiling-event slot recorded around this launch (-1: none)
   int ctas = 0;           // persistent CTAs: at most one per SM (0: as many as the GPU has SMs)
   bool streamk = false;   // stream-K schedule (one tile column; fp32 partial slabs reduced afterwards)
+  // launched as a programmatic dependent of the kernel before it in the stream: only where that kernel is this
+  // library's own and writes only what the GEMM reads after griddep_wait (the LoRA B operand)
+  bool pdl = false;
   UmmaArgs args{};
 };
+
+// Launch with programmatic stream serialization: the kernel may start while the one before it in the stream runs,
+// and waits for it (griddep_wait) before touching its outputs.
+template <typename Kern, typename... Args>
+cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 template <int BN, int AM, bool BMN, int KB = 1, bool PAIR = false, int WF = WF_NF4, int EPI = EPI_PLAIN>
 cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
@@ -295,7 +320,12 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
   } else {
     dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, g.ctas)));
     if (g.prof >= 0) prof_record(g.prof, 0, stream);
-    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmBx, tmC, g.args);
+    if (g.pdl && !prof_active(g.prof)) {
+      e = launch_dependent(kern, grid, dim3(C::kThreads), C::kSmemBytes, stream, tmA, tmB, tmBx, tmC, g.args);
+      if (e != cudaSuccess) return e;
+    } else {
+      kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmBx, tmC, g.args);
+    }
   }
   count_launch();
   if (g.prof >= 0) prof_record(g.prof, 1, stream);
@@ -508,13 +538,16 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass)
   return p;
 }
 
+// The split-K reduction of a GEMM's partials, launched as a dependent of that GEMM (it waits for it first).
 cudaError_t launch_reduce(const float* ws, int64_t slab, int nsplit, int64_t count, float alpha, void* out,
                           bool out_bf16, cudaStream_t stream) {
   if (count <= 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = std::min<int64_t>(cdiv(count, threads), 148 * 16);
-  reduce_splits_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(ws, slab, nsplit, count, alpha, out,
-                                                                              out_bf16 ? 1 : 0);
+  const cudaError_t e = launch_dependent(reduce_splits_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
+                                         stream, ws, static_cast<long long>(slab), nsplit,
+                                         static_cast<long long>(count), alpha, out, out_bf16 ? 1 : 0);
+  if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
 }
@@ -582,8 +615,11 @@ cudaError_t run_gemm(GemmCall g, void* out, bool out_bf16, float alpha, int64_t 
     if (e != cudaSuccess) return e;
     const int threads = 256;
     const int64_t blocks = std::min<int64_t>(cdiv(count, threads), 148 * 16);
-    reduce_streamk_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        part, count, count, cs, g.args.k_stages, T, g.ctas, alpha, out, out_bf16 ? 1 : 0);
+    e = launch_dependent(reduce_streamk_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream,
+                         static_cast<const float*>(part), static_cast<long long>(count), static_cast<long long>(count),
+                         static_cast<long long>(cs), static_cast<long long>(g.args.k_stages),
+                         static_cast<long long>(T), static_cast<long long>(g.ctas), alpha, out, out_bf16 ? 1 : 0);
+    if (e != cudaSuccess) return e;
     count_launch();
     return cudaGetLastError();
   }
@@ -739,6 +775,9 @@ ql_status linear_fwd_impl(int64_t M, int64_t N, int64_t K, int64_t r, const uint
     g.streamk = true;
     g.ctas = p.sk_ctas;
   }
+  // after this library's s x A^T kernels, the fused GEMM starts early: it reads their output (its LoRA B operand)
+  // and writes its own (which may share the workspace with their partials) only after griddep_wait
+  g.pdl = r > 0;
   g.prof = 0;
   if (epi) {
     g.args.epi = epi->mode;

@@ -181,6 +181,8 @@ __host__ __device__ __forceinline__ Unit sk_unit(const UmmaArgs& a, long long c,
 __global__ void reduce_streamk_kernel(const float* __restrict__ ws, long long slab, long long count, long long cs,
                                       long long S, long long T, long long P, float alpha, void* __restrict__ out,
                                       int out_bf16) {
+  griddep_launch_dependents();
+  griddep_wait();  // the slabs are the GEMM's output
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < count; e += stride) {
     const long long t = (e % cs) / 128;
@@ -457,12 +459,18 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
   if constexpr (PAIR) cluster_sync_all();  // the peer arrives on our barriers only once they exist
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a dependent of the kernel before it, this kernel reads nothing that kernel writes before the
+  // producer's griddep_wait (B of the LoRA stages in the dequantizing modes, every operand in the TMA modes), and
+  // writes nothing before the epilogue's; the weight codes and scales, the activations of the main stages and the
+  // LoRA rows come from before that kernel.
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ B producer
     Armed armed;
     int g = 0;
     bool stop = args.test_stall == 2;
+    bool dep_done = false;  // griddep_wait issued
     for (int u = first_unit; u < num_units && !stop; u += unit_step) {
       const Unit U = unit_of(args, u, BN, C::kPair, rank);
       for (int it = 0; it < U.n_total; ++it, ++g) {
@@ -474,6 +482,10 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
           break;
         }
         if (lane == 0) {
+          if (!dep_done && (!C::kDeq || it < U.n_extra)) {
+            griddep_wait();
+            dep_done = true;
+          }
           armed.set(s, ph);
           uint8_t* b_dst = sB + s * C::kBSlot;
           if constexpr (C::kDeq) {
@@ -608,6 +620,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
       tc_fence_after();
       ok = __shfl_sync(kFull, ok && !*abort_flag, 0);
       if (!ok) break;
+      if (lu == 0) griddep_wait();  // before the first global access of the epilogue
       const int i = U.i0 + qw * 32 + lane;
       const long long base = static_cast<long long>(U.z) * args.split_stride + static_cast<long long>(i) * args.ls;
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + static_cast<uint32_t>(acc * C::kAccCols);

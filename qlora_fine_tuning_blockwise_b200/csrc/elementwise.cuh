@@ -161,6 +161,37 @@ __global__ void nf4_dequantize_kernel(const uint8_t* __restrict__ codes, const f
   }
 }
 
+// su[m, j] = bf16(s * sum_k x[m, k] A[j, k]) for token-light layers (few outputs): one warp per output; lane l
+// accumulates in fp32 the products of its 8-element chunks 8 (l + 32 i) .. in order, then the lanes' sums combine
+// by a fixed butterfly.  Small CTAs with no shared memory fit beside a running fused GEMM; the GEMM that consumes su
+// may start at once (griddep_launch_dependents) and waits for this kernel before reading it.
+__global__ void su_small_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ A, int M, int K, int r,
+                                float s, uint16_t* __restrict__ su) {
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (w >= static_cast<long long>(M) * r) return;
+  const int m = static_cast<int>(w / r), j = static_cast<int>(w % r);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<long long>(m) * K);
+  const uint4* ar = reinterpret_cast<const uint4*>(A + static_cast<long long>(j) * K);
+  float acc = 0.0f;
+  for (int c = lane; c < K / 8; c += 32) {
+    const uint4 xv = __ldg(xr + c), av = __ldg(ar + c);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc = __fmaf_rn(__uint_as_float(xw[q] << 16), __uint_as_float(aw[q] << 16), acc);
+      acc = __fmaf_rn(__uint_as_float(xw[q] & 0xFFFF0000u), __uint_as_float(aw[q] & 0xFFFF0000u), acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+  if (lane == 0) {
+    const __nv_bfloat16 v = __float2bfloat16_rn(__fmul_rn(s, acc));
+    su[static_cast<long long>(m) * r + j] = *reinterpret_cast<const uint16_t*>(&v);
+  }
+}
+
 // out[e] = alpha * sum_s ws[s * slab + e]  (fp32 sum in split order: deterministic)
 __global__ void reduce_splits_kernel(const float* __restrict__ ws, long long slab, int nsplit, long long count,
                                      float alpha, void* __restrict__ out, int out_bf16) {

@@ -478,6 +478,9 @@ int plan_splits_streaming(int64_t tiles, int64_t kstages, int sms) {
 // dominate) when the absmax rows are whole 16-byte TMA boxes (K a multiple of 256), else 1.
 int fwd_stage_blocks(int64_t M, int64_t K) { return (main_bn(M) <= 64 && K % 256 == 0) ? 4 : 1; }
 
+// Token-light layers with few s x A^T outputs take them from CUDA cores (su_small_kernel).
+bool su_on_cores(int64_t M, int64_t r) { return M <= 64 && M * r <= 512; }
+
 struct LinearPlan {
   int bn_main = 16, s_main = 1;      // forward y / backward dX
   int sk_ctas = 0, sk_slabs = 0;     // stream-K forward: CTAs and partial slabs (0: split plan)
@@ -512,7 +515,7 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass)
   }
   if (p.s_main > 1) part = std::max(part, static_cast<size_t>(p.s_main) * M * (pass == QL_PASS_FWD ? N : K) * 4);
   if (r > 0) {
-    p.s_su = plan_splits(cdiv(M, 128) * (rp / rp), cdiv(K, 64), sms);
+    p.s_su = su_on_cores(M, r) ? 1 : plan_splits(cdiv(M, 128) * (rp / rp), cdiv(K, 64), sms);
     if (p.s_su > 1) part = std::max(part, static_cast<size_t>(p.s_su) * M * r * 4);
     if (pass == QL_PASS_BWD) {
       p.s_v = plan_splits(cdiv(M, 128), cdiv(N, 64), sms);
@@ -655,6 +658,14 @@ cudaError_t run_gemm(GemmCall g, void* out, bool out_bf16, float alpha, int64_t 
 // su = bf16(s * x A^T) [M, r]
 cudaError_t run_su(int64_t M, int64_t K, int64_t r, const uint16_t* x, const uint16_t* A, float s, uint16_t* su,
                    int splits, float* part, unsigned int* err, cudaStream_t stream) {
+  if (su_on_cores(M, r)) {
+    const int64_t warps = M * r;
+    su_small_kernel<<<static_cast<unsigned>(cdiv(warps, 2)), 64, 0, stream>>>(x, A, static_cast<int>(M),
+                                                                             static_cast<int>(K), static_cast<int>(r),
+                                                                             s, su);
+    count_launch();
+    return cudaGetLastError();
+  }
   GemmCall g;
   g.am = A_TMA_K;
   g.b_mn = false;
@@ -1456,7 +1467,8 @@ bool load_forward_kernels() {
          load_umma<32, A_DEQ_TMEM, false, 4>() && load_umma<64, A_DEQ_TMEM, false, 4>() &&
          load_umma<64, A_TMA_K, false>() && load_umma<128, A_TMA_K, false>() && load_umma<256, A_TMA_K, false>() &&
          cudaFuncGetAttributes(&a, reduce_splits_kernel) == cudaSuccess &&
-         cudaFuncGetAttributes(&a, reduce_streamk_kernel) == cudaSuccess;
+         cudaFuncGetAttributes(&a, reduce_streamk_kernel) == cudaSuccess &&
+         cudaFuncGetAttributes(&a, su_small_kernel) == cudaSuccess;
 }
 
 // Contexts in which the forward's kernels have been loaded (set-up runs once per context, with the device

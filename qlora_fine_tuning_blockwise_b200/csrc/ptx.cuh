@@ -96,6 +96,17 @@ __device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, v
   }
 }
 
+// ------------------------------------------------------------------------------------------ byte permute
+
+// prmt.b32 in its default mode: result byte i is byte (c >> 4i) & 7 of {b, a} (a = bytes 0..3), or -- when bit 3
+// of that selector nibble is set -- that byte's top bit replicated over all eight bits.  (__byte_perm reads only
+// the low three bits of each nibble.)
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // ------------------------------------------------------------------------------------------ dependent launch
 //
 // A kernel launched with programmatic stream serialization may start while the kernel before it in the stream is

@@ -816,6 +816,23 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
       const uint32_t t_lane = static_cast<uint32_t>(32 * (warp & 3)) << 16;
       const uint8_t* lut_lane = reinterpret_cast<const uint8_t*>(sLut) + lane * 4;
       const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+      // The MN-major (dX) dequantizer of NF4 codes looks levels up in registers instead of the shared table, which
+      // takes the table's 16 KB per stage off the shared-memory pipe that bounds dX: tl[q] / th[q] hold the low
+      // / high bytes of the bf16 levels 4q .. 4q + 3.
+      constexpr bool kRegTable = AM == A_DEQ_MN && WF != WF_NVFP4;
+      uint32_t tl[4] = {}, th[4] = {};
+      if constexpr (kRegTable) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat16 hv = __float2bfloat16_rn(kNF4LevelsDev[4 * q4 + e]);
+            const uint32_t bits = *reinterpret_cast<const uint16_t*>(&hv);
+            tl[q4] |= (bits & 0xFFu) << (8 * e);
+            th[q4] |= (bits >> 8) << (8 * e);
+          }
+        }
+      }
       const float dq_mu = WF == WF_NF4_DQ ? *args.dq_mu : 0.0f;
       const float fp4_S = WF == WF_NVFP4 ? *args.fp4_S : 0.0f;
       int g = 0, q = 0;
@@ -951,20 +968,47 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
                 }
                 sc2q[0] = sc2q[1] = sc2q[2] = sc2q[3] = __float2bfloat162_rn(a);
               }
+              if constexpr (kRegTable) {
+                // Per code word (8 elements; byte j holds element 2j in its high nibble): swap the nibbles of each
+                // byte so that nibble k is element k's code, select the level bytes of four codes at a time from
+                // the register table (codes 0..7 from tl[0..1], 8..15 from tl[2..3], chosen per byte by a mask of
+                // the codes' top bits, which prmt's sign mode spreads over their bytes), interleave low and high
+                // bytes into bf16 pairs, then scale.  Equal to the table lookup bit for bit.
 #pragma unroll
-              for (int w = 0; w < 8; ++w) {
-                const __nv_bfloat162 sc2 = sc2q[w >> 1];
-                const uint32_t qw8 = words[8 * p + w];
+                for (int w = 0; w < 8; ++w) {
+                  const __nv_bfloat162 sc2 = sc2q[w >> 1];
+                  const uint32_t qw8 = words[8 * p + w];
+                  const uint32_t qs = ((qw8 >> 4) & 0x0F0F0F0Fu) | ((qw8 << 4) & 0xF0F0F0F0u);
+                  const uint32_t s7 = qs & 0x77777777u, t4 = qs << 4;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  // byte offset of (code byte j, lane) in the table: one byte permute into (byte << 8) | 4 lane for
-                  // the wide table, a permute and a shift-add for the narrow one
-                  const uint32_t off =
-                      C::kWideLut ? __byte_perm(qw8, lane4, 0x5504u | (static_cast<uint32_t>(j) << 4))
-                                  : (__byte_perm(qw8, 0u, 0x4440u + static_cast<uint32_t>(j)) << 7) + lane4;
-                  uint32_t v = *reinterpret_cast<const uint32_t*>(smem_raw + off);
-                  __nv_bfloat162 pr = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc2);
-                  r[4 * w + j] = *reinterpret_cast<uint32_t*>(&pr);
+                  for (int hf = 0; hf < 2; ++hf) {
+                    const uint32_t sel = hf ? (s7 >> 16) : s7;
+                    const uint32_t m = prmt_sign(t4, qs, hf ? 0xFBEAu : 0xD9C8u);
+                    const uint32_t lo = (__byte_perm(tl[0], tl[1], sel) & ~m) | (__byte_perm(tl[2], tl[3], sel) & m);
+                    const uint32_t hi = (__byte_perm(th[0], th[1], sel) & ~m) | (__byte_perm(th[2], th[3], sel) & m);
+                    uint32_t v0 = __byte_perm(lo, hi, 0x5140u), v1 = __byte_perm(lo, hi, 0x7362u);
+                    const __nv_bfloat162 p0 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v0), sc2);
+                    const __nv_bfloat162 p1 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v1), sc2);
+                    r[4 * w + 2 * hf] = *reinterpret_cast<const uint32_t*>(&p0);
+                    r[4 * w + 2 * hf + 1] = *reinterpret_cast<const uint32_t*>(&p1);
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                  const __nv_bfloat162 sc2 = sc2q[w >> 1];
+                  const uint32_t qw8 = words[8 * p + w];
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    // byte offset of (code byte j, lane) in the table: one byte permute into (byte << 8) | 4 lane for
+                    // the wide table, a permute and a shift-add for the narrow one
+                    const uint32_t off =
+                        C::kWideLut ? __byte_perm(qw8, lane4, 0x5504u | (static_cast<uint32_t>(j) << 4))
+                                    : (__byte_perm(qw8, 0u, 0x4440u + static_cast<uint32_t>(j)) << 7) + lane4;
+                    uint32_t v = *reinterpret_cast<const uint32_t*>(smem_raw + off);
+                    __nv_bfloat162 pr = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc2);
+                    r[4 * w + j] = *reinterpret_cast<uint32_t*>(&pr);
+                  }
                 }
               }
             }

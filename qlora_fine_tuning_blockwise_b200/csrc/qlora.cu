@@ -220,7 +220,7 @@ cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t smem, cuda
 
 template <int BN, int AM, bool BMN, int KB = 1, bool PAIR = false, int WF = WF_NF4, int EPI = EPI_PLAIN>
 cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
-  using C = UmmaCfg<BN, AM, BMN, KB, PAIR, EPI>;
+  using C = UmmaCfg<BN, AM, BMN, KB, PAIR, EPI, WF>;
   CUtensorMap tmA, tmB, tmBx, tmC;
   std::memset(&tmA, 0, sizeof(tmA));
   std::memset(&tmBx, 0, sizeof(tmBx));

@@ -243,7 +243,7 @@ __device__ __forceinline__ Unit unit_of(const UmmaArgs& a, int u, int BN, int pa
 // barrier round trips of fixed latency, so token-light layers -- whose MMAs are short -- run 4 blocks a stage
 // (A_DEQ_TMEM only): codes then arrive as one 128B-swizzled TMA box of 128 rows x 128 bytes and the absmax
 // values as one TMA box of 128 rows x 4 floats.
-template <int BN, int AM, bool B_MN, int KB = 1, bool PAIR = false, int EPI = EPI_PLAIN>
+template <int BN, int AM, bool B_MN, int KB = 1, bool PAIR = false, int EPI = EPI_PLAIN, int WF = WF_NF4>
 struct UmmaCfg {
   static constexpr int kPair = PAIR ? 2 : 1;   // CTAs per MMA (cta_group::2: M = 256)
   static constexpr int kBRows = BN / kPair;    // B rows (tokens) held by each CTA
@@ -266,7 +266,9 @@ struct UmmaCfg {
   // kernel -- entry stride 256 bytes (64 KB, half of it padding), so that one byte permute of (code byte, lane)
   // is the whole offset
   static constexpr bool kWideLut = kDeq && KB == 4 && BN <= 32;
-  static constexpr int kLutBytes = kDeq ? (kWideLut ? 256 * 64 * 4 : 256 * 32 * 4) : 0;
+  // (the MN-major dequantizer of NF4 codes looks levels up in registers and needs no table)
+  static constexpr bool kRegTable = AM == A_DEQ_MN && WF != WF_NVFP4;
+  static constexpr int kLutBytes = (kDeq && !kRegTable) ? (kWideLut ? 256 * 64 * 4 : 256 * 32 * 4) : 0;
   static constexpr int kBarBytes = 1024;
   static constexpr int kBudget = 226 * 1024 - 1024 - kLutBytes - kBarBytes;
 
@@ -279,7 +281,8 @@ struct UmmaCfg {
 
   // ring depths: deep B rings when B tiles are small (token-light layers), 4 stages of 16-32 KB otherwise;
   // the A ring as deep as tensor memory (or shared memory, for A_DEQ_MN) allows.
-  static constexpr int kBStagesWant = kDeq ? (kWideLut ? 4 : BN <= 64 ? 8 : (AM == A_DEQ_MN && BN >= 256 ? 3 : 4)) : 8;
+  static constexpr int kBStagesWant =
+      kDeq ? (kWideLut ? 4 : BN <= 64 ? 8 : (AM == A_DEQ_MN && BN >= 256 ? (kRegTable ? 4 : 3) : 4)) : 8;
   static constexpr int kAStagesWant = kATmem ? kAStagesTmem : (AM == A_DEQ_MN ? (BN >= 256 ? 3 : 4) : 0);
   static constexpr int kQWant = KB == 4 ? 6 : (BN >= 128 ? 10 : 16);
   static constexpr int kBFit = (kBudget - kAStagesWant * kASlot - (kDeq ? kQWant * kQSlot : 0)) / kBSlot;
@@ -350,11 +353,11 @@ struct Armed {
 
 // tmA: A for the TMA modes; the absmax matrix [w_rows, w_cols / 64] (fp32) for 4-block TMEM stages.
 template <int BN, int AM, bool B_MN, int KB = 1, bool PAIR = false, int WF = WF_NF4, int EPI = EPI_PLAIN>
-__global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads, 1)
+__global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC,
                      const UmmaArgs args) {
-  using C = UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>;
+  using C = UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>;
   static_assert(AM != A_DEQ_TMEM_T || WF == WF_NF4, "the transposed TMEM dequantizer reads NF4 weights");
   constexpr int BS = C::kBStages;
   constexpr int AS = C::kAStages;
@@ -819,9 +822,8 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
       // The MN-major (dX) dequantizer of NF4 codes looks levels up in registers instead of the shared table, which
       // takes the table's 16 KB per stage off the shared-memory pipe that bounds dX: tl[q] / th[q] hold the low
       // / high bytes of the bf16 levels 4q .. 4q + 3.
-      constexpr bool kRegTable = AM == A_DEQ_MN && WF != WF_NVFP4;
       uint32_t tl[4] = {}, th[4] = {};
-      if constexpr (kRegTable) {
+      if constexpr (C::kRegTable) {
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
 #pragma unroll
@@ -968,7 +970,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI>::kThreads
                 }
                 sc2q[0] = sc2q[1] = sc2q[2] = sc2q[3] = __float2bfloat162_rn(a);
               }
-              if constexpr (kRegTable) {
+              if constexpr (C::kRegTable) {
                 // Per code word (8 elements; byte j holds element 2j in its high nibble): swap the nibbles of each
                 // byte so that nibble k is element k's code, select the level bytes of four codes at a time from
                 // the register table (codes 0..7 from tl[0..1], 8..15 from tl[2..3], chosen per byte by a mask of

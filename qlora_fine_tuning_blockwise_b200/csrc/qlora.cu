@@ -119,9 +119,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major matrix [rows, cols] of 1-, 2- or 4-byte elements; box = box_cols x box_rows.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
-              int box_rows, bool swizzle128) {
+// Row-major matrix [rows, cols] of 1-, 2- or 4-byte elements; box = box_cols x box_rows, written to shared
+// memory with the given swizzle (a box row of 32, 64 or 128 bytes has its 16-byte chunk c at c XOR bits 7.. of its
+// shared-memory address).
+bool make_map_sw(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
+                 int box_rows, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -132,10 +134,15 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
                                  : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                    : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUresult r = fn(m, dt, 2,
-                  const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
+              int box_rows, bool swizzle128) {
+  return make_map_sw(m, base, rows, cols, elem_bytes, box_cols, box_rows,
+                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // ------------------------------------------------------------------------------------------ GEMM launch
@@ -256,8 +263,12 @@ cudaError_t launch_umma(const GemmCall& g, cudaStream_t stream) {
     }
   } else if (C::kDeq) {
     const int64_t N = g.args.w_rows, K = g.args.w_cols;
+    // codes rows of 32 bytes (forward) or 64 bytes (dX) swizzled so that the dequantizers' 16-byte loads of
+    // eight consecutive rows hit eight distinct bank groups; the transposing dequantizer reads single bytes
     if (AM == A_DEQ_TMEM) {
-      if (!make_map(&tmC, g.codes, N, K / 2, 1, 32, 128, false)) return cudaErrorInvalidValue;
+      if (!make_map_sw(&tmC, g.codes, N, K / 2, 1, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return cudaErrorInvalidValue;
+    } else if (AM == A_DEQ_MN) {
+      if (!make_map_sw(&tmC, g.codes, N, K / 2, 1, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B)) return cudaErrorInvalidValue;
     } else {
       if (!make_map(&tmC, g.codes, N, K / 2, 1, 64, 64, false)) return cudaErrorInvalidValue;
     }

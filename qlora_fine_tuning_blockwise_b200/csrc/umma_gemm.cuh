@@ -814,7 +814,6 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
       //             map so that the 8 lanes of a store phase hit 8 distinct 16-byte bank groups.
       const int row = C::kATmem ? 32 * (warp & 3) + lane : ((tg & 7) + 8 * (tg >> 4));
       const int h = C::kATmem ? 0 : ((tg >> 3) & 1);
-      const int c_off = C::kATmem ? row * 32 : (row * 64 + h * 32);
       const int s_idx = C::kATmem ? row : (row * 2 + h);
       const uint32_t t_lane = static_cast<uint32_t>(32 * (warp & 3)) << 16;
       const uint8_t* lut_lane = reinterpret_cast<const uint8_t*>(sLut) + lane * 4;
@@ -896,8 +895,13 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
               }
             } else {
               sw[0] = reinterpret_cast<const uint32_t*>(q_src + C::kCBytes)[s_idx];
-              const uint4 c01 = *reinterpret_cast<const uint4*>(q_src + c_off);
-              const uint4 c23 = *reinterpret_cast<const uint4*>(q_src + c_off + 16);
+              // the thread's two 16-byte chunks (c0, c0 + 1) of its codes row, each at its swizzled position:
+              // 32-byte rows (forward) XOR bit 7 of the address, 64-byte rows (dX) XOR bits 7..8
+              const int c0 = C::kATmem ? 0 : 2 * h;
+              const int sx = C::kATmem ? ((row >> 2) & 1) : ((row >> 1) & 3);
+              const uint8_t* q_row = q_src + (C::kATmem ? row * 32 : row * 64);
+              const uint4 c01 = *reinterpret_cast<const uint4*>(q_row + ((c0 ^ sx) << 4));
+              const uint4 c23 = *reinterpret_cast<const uint4*>(q_row + (((c0 + 1) ^ sx) << 4));
               words[0] = c01.x;
               words[1] = c01.y;
               words[2] = c01.z;

@@ -37,27 +37,39 @@ struct Nf4Thresholds {
   }
 };
 
-// One warp per 64-element block: lane l owns elements 2l, 2l+1 (one packed byte).
+// One warp per 64-element block: lane l owns elements 2l, 2l+1 (one packed byte).  A warp takes four consecutive
+// blocks per step and issues their loads before it works on any of them, so four 8-byte loads per lane are in
+// flight instead of one.
+constexpr int kQuantBlocksPerStep = 4;
+
 __global__ void nf4_quantize_kernel(const float* __restrict__ w, long long nblocks, uint8_t* __restrict__ codes,
                                     float* __restrict__ absmax, unsigned int* err) {
   const int lane = threadIdx.x & 31;
   const Nf4Thresholds thr;
   const long long warps_total = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  for (long long b = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); b < nblocks;
-       b += warps_total) {
-    const float2 v = __ldg(reinterpret_cast<const float2*>(w) + b * 32 + lane);
-    float m = fmaxf(fabsf(v.x), fabsf(v.y));
+  const long long warp_id = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  for (long long b0 = warp_id * kQuantBlocksPerStep; b0 < nblocks; b0 += warps_total * kQuantBlocksPerStep) {
+    float2 v[kQuantBlocksPerStep];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const bool bad = !isfinite(v.x) || !isfinite(v.y);
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, kDevErrNonFinite);
-    uint32_t c0 = 7, c1 = 7;
-    if (m > 0.0f) {
-      c0 = thr.code(__fdiv_rn(v.x, m));
-      c1 = thr.code(__fdiv_rn(v.y, m));
+    for (int i = 0; i < kQuantBlocksPerStep; ++i)
+      v[i] = b0 + i < nblocks ? __ldg(reinterpret_cast<const float2*>(w) + (b0 + i) * 32 + lane) : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kQuantBlocksPerStep; ++i) {
+      const long long b = b0 + i;
+      if (b >= nblocks) break;  // warp-uniform
+      float m = fmaxf(fabsf(v[i].x), fabsf(v[i].y));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const bool bad = !isfinite(v[i].x) || !isfinite(v[i].y);
+      if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, kDevErrNonFinite);
+      uint32_t c0 = 7, c1 = 7;
+      if (m > 0.0f) {
+        c0 = thr.code(__fdiv_rn(v[i].x, m));
+        c1 = thr.code(__fdiv_rn(v[i].y, m));
+      }
+      codes[b * 32 + lane] = static_cast<uint8_t>((c0 << 4) | c1);
+      if (lane == 0) absmax[b] = m;
     }
-    codes[b * 32 + lane] = static_cast<uint8_t>((c0 << 4) | c1);
-    if (lane == 0) absmax[b] = m;
   }
 }
 

@@ -1060,8 +1060,9 @@ ql_status nf4_quantize(const float* w, int64_t numel, int blocksize, uint8_t* co
   DeviceInfo d;
   if (!device_info(&d)) return QL_ERR_CUDA;
   const long long nblocks = numel / 64;
-  const int threads = 256;  // 8 warps = 8 blocks per CTA iteration
-  const long long ctas = std::min<long long>(cdiv(nblocks, 8), static_cast<long long>(d.sms) * 32);
+  const int threads = 256;  // 8 warps, each taking kQuantBlocksPerStep blocks per step
+  const long long ctas =
+      std::min<long long>(cdiv(nblocks, 8 * kQuantBlocksPerStep), static_cast<long long>(d.sms) * 16);
   nf4_quantize_kernel<<<static_cast<unsigned>(ctas), threads, 0, as_stream(stream)>>>(w, nblocks, codes, absmax, d.err);
   count_launch();
   return status_of(cudaGetLastError());

@@ -920,6 +920,9 @@ ql_status linear_bwd_impl(int64_t M, int64_t N, int64_t K, int64_t r, const uint
     g.k_total = N;
     g.splits = p.s_main;
     g.prof = 1;
+    // after this library's v kernels, dX starts early: it reads v (its LoRA B operand, in the stages after its
+    // first unit's main stages) and writes its output only after griddep_wait
+    g.pdl = r > 0;
     if (epi) {
       g.args.epi = epi->mode;
       g.args.out2 = epi->out2;

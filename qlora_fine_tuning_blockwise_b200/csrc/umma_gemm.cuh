@@ -1,10 +1,11 @@
 // tcgen05 GEMM kernel for the QLoRA layer (sm_100a), persistent over work units.
 //
 // A work unit is a 128 x BN fp32 tile of D[i, j] = sum_kk Aop[i, kk] * Bop[j, kk] accumulated in TMEM over
-// one split of the contraction (stages of KB blocks of 64 elements), optionally preceded by "extra" stages
-// that append the
-// rank-r LoRA columns to the contraction ([x | s u] . [deq(W) | B]^T in the forward, [dY | v] . [deq(W); A]
-// in the backward), so base and LoRA products land in one accumulator.  Each CTA walks units
+// one split of the contraction (stages of KB blocks of 64 elements), optionally followed by "extra" stages that
+// append the rank-r LoRA columns to the contraction ([x | s u] . [deq(W) | B]^T in the forward, [dY | v] .
+// [deq(W); A] in the backward), so base and LoRA products land in one accumulator.  The LoRA stages come last so
+// that a kernel launched as a dependent of the one computing s u (or v) needs that operand only at the end of
+// its first unit.  Each CTA walks units
 // blockIdx.x, blockIdx.x + gridDim.x, ...; its rings run on across units, and where tensor memory allows
 // two accumulators alternate between units so the epilogue of one overlaps the mainloop of the next.
 //
@@ -88,7 +89,7 @@ struct UmmaArgs {
   int splits;             // contraction splits; units = splits * tiles_i * tiles_j
   int k_stages;           // main contraction stages (64 KB elements each) in total
   int stages_per_split;   // main stages per split
-  int n_extra;            // extra (LoRA) stages, run by split 0 only, before its main stages
+  int n_extra;            // extra (LoRA) stages, run by split 0 only, after its main stages
   // dequantization (A_DEQ_*): W is [w_rows, w_cols] of packed 4-bit codes in format `wfmt` with one 4-byte
   // scale word per 64-element block, `scale_words` [w_rows, w_cols / 64]:
   //   WF_NF4    : the fp32 absmax of the block (codes: NF4 levels, element 2j in the high nibble);
@@ -158,7 +159,8 @@ __host__ __device__ __forceinline__ int sk_units(const UmmaArgs& a, long long c,
 }
 
 // Stream-K: unit u of CTA c of P -- the part of tile s0 / S + u inside the CTA's share, its slab z (the CTA's
-// place among those sharing the tile) and, for the part that starts the tile, the LoRA stages.
+// place among those sharing the tile) and, for the part that starts the tile, the LoRA stages (that part is the
+// last unit of its CTA, so the LoRA operand is needed only at the end of the CTA's work).
 __host__ __device__ __forceinline__ Unit sk_unit(const UmmaArgs& a, long long c, long long P, int u) {
   Unit U;
   const long long S = a.sk_stages, T = static_cast<long long>(a.tiles_i) * S;
@@ -485,7 +487,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
           break;
         }
         if (lane == 0) {
-          if (!dep_done && (!C::kDeq || it < U.n_extra)) {
+          if (!dep_done && (!C::kDeq || it >= U.n_main)) {
             griddep_wait();
             dep_done = true;
           }
@@ -499,8 +501,9 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
 #pragma unroll
             for (int kb = 0; kb < KB; ++kb) {
               uint8_t* dst = b_dst + kb * C::kBRows * 128;
-              const int x = it < U.n_extra ? 64 * (KB * it + kb) : ((U.main_begin + it - U.n_extra) * KB + kb) * 64;
-              const CUtensorMap* tm = it < U.n_extra ? &tmBx : &tmB;
+              const bool ex = it >= U.n_main;  // the LoRA stages follow the unit's main stages
+              const int x = ex ? 64 * (KB * (it - U.n_main) + kb) : ((U.main_begin + it) * KB + kb) * 64;
+              const CUtensorMap* tm = ex ? &tmBx : &tmB;
               if constexpr (PAIR)
                 tma_load_2d_pair(dst, tm, x, jb, &b_full[s]);
               else
@@ -744,7 +747,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
       bool stop = args.test_stall == 3;
       for (int u = first_unit; u < num_units && !stop; u += unit_step) {
         const Unit U = unit_of(args, u, BN, C::kPair, rank);
-        for (int it = U.n_extra; it < U.n_total; ++it, ++q) {
+        for (int it = 0; it < U.n_main; ++it, ++q) {
           const int s = q % QS;
           const uint32_t ph = static_cast<uint32_t>(q / QS) & 1u;
           const bool ok = mbar_wait_idle(&q_empty[s], ph ^ 1u, abort_flag, args.err, lim);
@@ -752,7 +755,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
             stop = true;
             break;
           }
-          const int kk0 = (U.main_begin + it - U.n_extra) * 64 * KB;
+          const int kk0 = (U.main_begin + it) * 64 * KB;
           uint8_t* q_dst = sQ + s * C::kQSlot;
           // 4-block stages take their scale words by TMA, except the double-quantized constants (4 bytes a row,
           // below the 16-byte minimum of a TMA box row)
@@ -841,7 +844,8 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
       for (int u = first_unit; u < num_units && !stop; u += unit_step) {
         const Unit U = unit_of(args, u, BN, C::kPair, rank);
         for (int it = 0; it < U.n_total; ++it, ++g) {
-          const bool extra = it < U.n_extra;
+          const bool extra = it >= U.n_main;
+          const int xe = it - U.n_main;  // LoRA stage index within the unit
           const int qi = q;
           if (!extra) ++q;
           if (g % C::kDeqGroups != grp) continue;
@@ -926,11 +930,11 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
               int c0 = 0;
               if constexpr (C::kATmem) {
                 const int n = U.i0 + row;
-                c0 = 64 * (KB * it + p);
+                c0 = 64 * (KB * xe + p);
                 valid = n < args.w_rows;
                 src = args.lora + static_cast<long long>(n) * args.lora_ld + c0;
               } else {
-                const int jr = 64 * it + row;
+                const int jr = 64 * xe + row;
                 valid = jr < args.lora_r && U.i0 + 64 * h < args.w_cols;
                 src = args.lora + static_cast<long long>(jr) * args.lora_ld + U.i0 + 64 * h;
               }
@@ -958,9 +962,9 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
                   int n, kb;
                   if constexpr (C::kATmem) {
                     n = U.i0 + row;
-                    kb = (U.main_begin + it - U.n_extra) * KB + p;
+                    kb = (U.main_begin + it) * KB + p;
                   } else {
-                    n = (U.main_begin + it - U.n_extra) * 64 + row;
+                    n = (U.main_begin + it) * 64 + row;
                     kb = (U.i0 >> 6) + h;
                   }
                   const long long blk = static_cast<long long>(n) * args.w_kb + kb;
@@ -1026,7 +1030,7 @@ __global__ void __launch_bounds__(UmmaCfg<BN, AM, B_MN, KB, PAIR, EPI, WF>::kThr
               const bool vk = k < args.w_cols;
 #pragma unroll
               for (int pp = 0; pp < 32; ++pp) {
-                const int j = 64 * it + 2 * pp;
+                const int j = 64 * xe + 2 * pp;
                 const uint32_t lo = (vk && j < args.lora_r)
                                         ? __ldg(args.lora + static_cast<long long>(j) * args.lora_ld + k) : 0u;
                 const uint32_t hi = (vk && j + 1 < args.lora_r)

@@ -101,11 +101,12 @@ def make_world(cfg, seed):
 
 
 def stages(cfg):
-    """(global stage g, main index q or None, unit index, index within the unit) in issue order."""
+    """(global stage g, main index q or None, unit index, index within the unit) in issue order: a unit's main
+    stages, then its extra (LoRA) stages, as the kernel issues them."""
     out, g, q = [], 0, 0
     for ui, (ne, nm) in enumerate(cfg.units):
         for it in range(ne + nm):
-            main = it >= ne
+            main = it < nm
             out.append((g, q if main else None, ui, it))
             g += 1
             if main:

@@ -149,8 +149,8 @@ QL_API ql_status qlora_merge_lora_nf4(int64_t N, int64_t K, int64_t r, const uin
 
 /*
  * qlora_workspace_bytes -- device scratch needed by qlora_linear_fwd (pass = QL_PASS_FWD) or
- * qlora_linear_bwd (QL_PASS_BWD) for these sizes on the current device (split-K partial sums, the
- * rank-r intermediates s*x*A^T and s*dY*B).  Host-only.  Returns 0 when nothing is needed.
+ * qlora_linear_bwd (QL_PASS_BWD) for these sizes on the current device (split-K or stream-K partial sums,
+ * the rank-r intermediates s*x*A^T and s*dY*B).  Host-only.  Returns 0 when nothing is needed.
  */
 QL_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass);
 

@@ -104,7 +104,34 @@ __global__ void lora_merge_kernel(const uint8_t* __restrict__ codes, const float
     float acc0 = 0.0f, acc1 = 0.0f;
     const uint16_t* brow = B + n * r;
     const uint32_t* apair = reinterpret_cast<const uint32_t*>(A + k0) + lane;  // A[j, k0 + 2l .. k0 + 2l + 1]
-    for (int j = 0; j < r; ++j) {
+    // eight ranks at a time: their loads are issued together (one 16-byte load of B's row when r is a multiple
+    // of 8, so the row is 16-byte aligned), then summed in the same order, one rank after the other
+    const int r8 = r & ~7;
+    int j = 0;
+    for (; j < r8; j += 8) {
+      uint32_t bw[4];
+      if ((r & 7) == 0) {
+        const uint4 b8 = __ldg(reinterpret_cast<const uint4*>(brow + j));
+        bw[0] = b8.x;
+        bw[1] = b8.y;
+        bw[2] = b8.z;
+        bw[3] = b8.w;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          bw[q] = static_cast<uint32_t>(__ldg(brow + j + 2 * q)) | (static_cast<uint32_t>(__ldg(brow + j + 2 * q + 1)) << 16);
+      }
+      uint32_t a8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) a8[q] = __ldg(apair + static_cast<long long>(j + q) * (K / 2));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float bj = __uint_as_float((q & 1) ? (bw[q >> 1] & 0xFFFF0000u) : (bw[q >> 1] << 16));
+        acc0 = __fadd_rn(acc0, __fmul_rn(bj, __uint_as_float(a8[q] << 16)));
+        acc1 = __fadd_rn(acc1, __fmul_rn(bj, __uint_as_float(a8[q] & 0xFFFF0000u)));
+      }
+    }
+    for (; j < r; ++j) {
       const float bj = __uint_as_float(static_cast<uint32_t>(__ldg(brow + j)) << 16);
       const uint32_t a = __ldg(apair + static_cast<long long>(j) * (K / 2));
       acc0 = __fadd_rn(acc0, __fmul_rn(bj, __uint_as_float(a << 16)));

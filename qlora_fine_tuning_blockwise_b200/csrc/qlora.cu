@@ -527,6 +527,14 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int64_t r, ql_pass pass)
   if (p.s_main > 1) part = std::max(part, static_cast<size_t>(p.s_main) * M * (pass == QL_PASS_FWD ? N : K) * 4);
   if (r > 0) {
     p.s_su = su_on_cores(M, r) ? 1 : plan_splits(cdiv(M, 128) * (rp / rp), cdiv(K, 64), sms);
+    if (pass == QL_PASS_FWD && !su_on_cores(M, r) && p.sk_slabs == 0) {
+      // The fused GEMM starts while s x A^T runs; its CTAs on the SMs that s x A^T holds start late.  When the
+      // unsplit s x A^T needs no more CTAs than the fused GEMM has CTAs with one unit fewer than the rest, those
+      // late CTAs are exactly the short ones and the fused GEMM ends no later: run s x A^T unsplit.
+      const int64_t units = main_tiles * p.s_main;
+      const int64_t short_ctas = units % sms == 0 ? 0 : sms - units % sms;
+      if (units > sms && cdiv(M, 128) <= short_ctas) p.s_su = 1;
+    }
     if (p.s_su > 1) part = std::max(part, static_cast<size_t>(p.s_su) * M * r * 4);
     if (pass == QL_PASS_BWD) {
       p.s_v = plan_splits(cdiv(M, 128), cdiv(N, 64), sms);

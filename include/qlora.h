@@ -89,8 +89,8 @@ QL_API ql_status ql_selftest_wait_timeout(int64_t wait_cycles, void* stream);
  * then has a copy or an MMA in flight.  Every wait of that launch is bounded by wait_cycles (>= 100000) instead
  * of about 2 s, so the other roles' waits expire: the kernel raises its abort flag, drains the copies it issued,
  * frees its tensor memory and returns; ql_get_device_error then reports QL_ERR_TIMEOUT and the call's outputs
- * are undefined.  Role 3 with r > 0 lets the LoRA stages reach the MMA before the stall, so use it with r = 0.
- * The arming is consumed by that one launch.
+ * are undefined.  (A unit's LoRA stages follow its main stages, so with role 3 no stage of the first unit is ever
+ * complete, whatever the rank.)  The arming is consumed by that one launch.
  */
 QL_API ql_status ql_selftest_arm_gemm_stall(int role, int64_t wait_cycles);
 

@@ -15,9 +15,10 @@ Modules
 
 Pins: every function here is checked by ``tests/test_oracle_*.py`` against values fixed by the
 mathematics (closed forms, invariants, brute force on tiny inputs, finite differences, library routines
-for the special cases that reduce to them).  The one part with no external pin is the exact NF4 table:
-the pages name the level set but print no table ("parity unpinned" against the pages for the table
-values; see ``oracle.nf4.nf4_codebook``).
+for the special cases that reduce to them).  The exact NF4 table, which the pages name but do not print, is
+pinned to the sixteen values printed in the paper that defines NF4 (QLoRA: Efficient Finetuning of Quantized
+LLMs, Appendix E, "NormalFloat 4-bit data type"), kept as text in ``tests/golden/nf4_qlora_paper.txt`` and checked
+by ``tests/test_oracle_nf4.py``.
 """
 
 from . import nf4, linear, merge, double_quant, nvfp4  # noqa: F401

@@ -3,6 +3,8 @@
 // every stage of every tile is done exactly once, a tile's parts come from consecutive CTAs in stage order with
 // slabs z = 0, 1, ..., the part count equals what the reduction sums, the LoRA stages run once per tile (in slab
 // 0), and every CTA gets floor or ceil of T / P stages.  Prints one line per case: "ok ..." or "FAIL ...".
+// With the argument "planted" the last CTA walks the schedule of a grid one CTA larger (a plausible mistake: the
+// grid size and the P the schedule assumes disagree); every case must then fail.
 #include <cstdio>
 #include <cstdlib>
 #include <vector>
@@ -10,6 +12,8 @@
 #include "../qlora_fine_tuning_blockwise_b200/csrc/umma_gemm.cuh"
 
 using namespace qlora;
+
+static bool g_planted = false;
 
 static bool check(int tiles, int S, int P, int n_extra) {
   UmmaArgs a{};
@@ -20,9 +24,10 @@ static bool check(int tiles, int S, int P, int n_extra) {
   std::vector<int> done(T, 0), extra(tiles, 0), parts(tiles, 0), last_cta(tiles, -1), next_stage(tiles, 0);
   for (int c = 0; c < P; ++c) {
     long long work = 0;
-    const int n = sk_units(a, c, P);
+    const long long Pc = (g_planted && c == P - 1) ? P + 1 : P;
+    const int n = sk_units(a, c, Pc);
     for (int u = 0; u < n; ++u) {
-      const Unit U = sk_unit(a, c, P, u);
+      const Unit U = sk_unit(a, c, Pc, u);
       const int t = U.i0 / 128;
       if (t < 0 || t >= tiles || U.n_main <= 0 || U.main_begin != next_stage[t] || U.z != parts[t] ||
           (last_cta[t] >= 0 && last_cta[t] != c - 1)) {
@@ -63,7 +68,8 @@ static bool check(int tiles, int S, int P, int n_extra) {
   return true;
 }
 
-int main() {
+int main(int argc, char** argv) {
+  g_planted = argc > 1 && argv[1][0] == 'p';
   bool all = true;
   all &= check(224, 32, 148, 1);   // 16 tokens x 8192 -> 28672, four-block stages
   all &= check(8, 16, 32, 1);
@@ -79,6 +85,9 @@ int main() {
     const long long T = static_cast<long long>(tiles) * S;
     const int P = 1 + static_cast<int>(std::rand() % (T < 148 ? T : 148));
     all &= check(tiles, S, P, std::rand() % 3);
+  }
+  if (g_planted) {  // every case must have failed
+    return all ? 1 : 0;
   }
   return all ? 0 : 1;
 }

@@ -3,7 +3,8 @@
 tests/streamk_schedule.cu compiles the kernel's own schedule functions for the host and walks them over the
 decode layer's shape and a few hundred random (tiles, stages per tile, CTAs): every stage of every tile is done
 once, a tile's parts come from consecutive CTAs in order with slabs 0, 1, ... -- as many as the reduction sums --,
-the LoRA stages run once per tile, and the CTAs' stage counts differ by at most one.
+the LoRA stages run once per tile, and the CTAs' stage counts differ by at most one.  A planted mistake (one CTA
+walking the schedule of a grid one CTA larger) must make every case fail.
 """
 
 import os
@@ -25,3 +26,7 @@ def test_streamk_schedule_is_a_balanced_partition(tmp_path):
     lines = r.stdout.strip().splitlines()
     assert r.returncode == 0, [l for l in lines if l.startswith("FAIL")][:5]
     assert len(lines) == 308 and all(l.startswith("ok ") for l in lines)
+    # the checker catches a schedule walked with the wrong grid size on one CTA
+    r = subprocess.run([exe, "planted"], capture_output=True, text=True)
+    lines = r.stdout.strip().splitlines()
+    assert r.returncode == 0 and not any(l.startswith("ok ") for l in lines), [l for l in lines if l.startswith("ok")][:3]

@@ -102,6 +102,17 @@ def test_workspace_plan_is_host_only_and_sane(L):
     assert L.workspace_bytes(0, 4096, 4096, 16, L.QL_PASS_FWD) == 0
 
 
+def test_forward_splits_s_x_at_only_where_the_fused_gemm_cannot_absorb_it(L):
+    """The forward plan (for 148 SMs, the host-side default) runs s x A^T unsplit -- no fp32 partial sums in the
+    workspace -- when its CTAs fit on the fused GEMM's CTAs that own one unit fewer (the attention layer: 256 units,
+    40 short CTAs, 16 s x A^T CTAs; the MLP down projection: 512 units, 80 short, 32), and splits it where every CTA
+    of the fused GEMM carries the same load (the block's layers)."""
+    assert L.workspace_bytes(2048, 4096, 4096, 16, L.QL_PASS_FWD) == 2048 * 16 * 2
+    assert L.workspace_bytes(4096, 4096, 11008, 64, L.QL_PASS_FWD) == 4096 * 64 * 2
+    assert L.workspace_bytes(8192, 57344, 8192, 128, L.QL_PASS_FWD) > 8192 * 128 * 2
+    assert L.workspace_bytes(8192, 8192, 28672, 64, L.QL_PASS_FWD) > 8192 * 64 * 2
+
+
 def test_swiglu_rejects_bad_arguments_on_host(L):
     lib = L.lib()
     p = ctypes.c_void_p(FAKE)
